@@ -1,0 +1,397 @@
+"""Benchmark of the B200 MLA-absorb tree-verify attention.
+
+One step = one verify call (split kernel + LSE-merge reduce) over the
+65k-context workload: 1 request, 64 heads, a 64-node random tree (depth
+<= 16), 65,536-token prefix, scattered slots in a 262,144-slot bf16 latent
+pool. The call is captured in CUDA graphs with a static workspace and
+replayed; L2 is flushed (256 MiB write) before every timed step and the
+flush is outside the timed events.
+
+Prints one JSON line (rank 0). ``value`` is KV tokens per second (sum of the
+requests' KV lengths per call / device time per call), whole job over all
+ranks; ``--gpus N`` runs N independent replicas (the path needs no
+collective). ``--impl reference`` times the float64 CPU oracle instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, generate  # noqa: E402
+
+METRIC = "tree-verify attn µs/call, KV tok/s & HBM GB/s (% roofline) at 65k ctx"
+UNIT = "KV tok/s"
+WORKLOAD = "long"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_config(wl, extra=None):
+    cfg = {
+        "workload": "long: 1 request, H=64 heads, T=64 random tree (depth<=16), prefix L=65536, "
+                    "q_latent 512 + q_rope 64, c_kv 512 + k_rope 64 bf16, scattered slots in a "
+                    "262144-slot page_size=1 pool, scale 192^-0.5",
+        "batch": wl.batch, "num_heads": wl.num_heads, "tree_nodes": list(wl.tree_sizes),
+        "prefix": list(wl.prefixes), "kv_per_call": wl.total_kv, "pool_slots": wl.pool_slots,
+        "kv_layout": wl.layout, "l2": "flushed before every timed step (256 MiB write, outside the events)",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(inp, anc):
+    """(flops, bytes) the method must do: every visible (row, key) pair costs
+    2*(576+512) flops; every KV row, q row and output row moves once."""
+    H = inp.q_latent.shape[1]
+    visible = 0
+    for b in range(len(inp.qo_indptr) - 1):
+        q0, q1 = int(inp.qo_indptr[b]), int(inp.qo_indptr[b + 1])
+        L = int(inp.kv_indptr[b + 1] - inp.kv_indptr[b]) - (q1 - q0)
+        visible += sum(L + bin(int(a)).count("1") for a in anc[q0:q1])
+    rows = inp.q_latent.shape[0] * H
+    total_kv = int(inp.kv_indptr[-1])
+    flops = 2.0 * H * visible * (576 + 512)
+    nbytes = total_kv * 1152 + rows * 1152 + rows * 1024 + total_kv * 4
+    return flops, nbytes
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            lines = open(self.path).read().strip().splitlines()
+        except OSError:
+            lines = []
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if self.path:
+            os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(inp, anc_oracle, budget_s: float = 12.0):
+    """Time the float64 oracle on whole query rows of the same workload until
+    about `budget_s` seconds of work are done; scale to the full call."""
+    import oracle
+
+    H = inp.q_latent.shape[1]
+    rows_total = inp.q_latent.shape[0] * H
+    cores = len(os.sched_getaffinity(0))
+    order = np.random.default_rng(0).permutation(rows_total).astype(np.int64)
+    chunk = max(cores, 1)
+    done, t0 = 0, time.perf_counter()
+    while done < rows_total and time.perf_counter() - t0 < budget_s:
+        oracle.verify_rows(inp, anc_oracle, rows=order[done:done + chunk], threads=cores)
+        done += chunk
+        chunk = min(chunk * 2, rows_total - done) if done < rows_total else chunk
+    elapsed = time.perf_counter() - t0
+    full_call_s = elapsed * rows_total / done
+    value = int(inp.kv_indptr[-1]) / full_call_s
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {rows_total} (token, head) query rows of the {WORKLOAD} workload, each over its "
+                      f"full 65.6k-key visible set, float64 C oracle with OpenMP; {elapsed:.1f} s scaled to the "
+                      f"full call by rows"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    wl = WORKLOADS[WORKLOAD]
+    inp = generate(wl)
+    anc = oracle.ancestor_masks(inp.parents, inp.qo_indptr)
+    H = inp.q_latent.shape[1]
+    rows_total = inp.q_latent.shape[0] * H
+    cores = len(os.sched_getaffinity(0))
+    rows_per_step = max(cores, 8)
+    order = np.random.default_rng(1).permutation(rows_total).astype(np.int64)
+    pos = 0
+
+    def step():
+        nonlocal pos
+        sel = order[pos:pos + rows_per_step]
+        if sel.shape[0] < rows_per_step:
+            pos = 0
+            sel = order[:rows_per_step]
+        pos += rows_per_step
+        oracle.verify_rows(inp, anc, rows=sel, threads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    elapsed = time.perf_counter() - t0
+    per_call = elapsed / args.steps * rows_total / rows_per_step
+    value = wl.total_kv / per_call
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, {"step": f"{rows_per_step} query rows of {rows_total} per step"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_per_step} of {rows_total} query rows per step, scaled by rows"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args):
+    import torch
+
+    import mla_speculative_verify_absorb_b200 as va
+    from workloads import device as wdev
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    wl = WORKLOADS[WORKLOAD]
+    inp = generate(wl)
+    anc = np.concatenate([va.verify_attn_build_tree_mask(inp.parents[int(inp.qo_indptr[b]):int(inp.qo_indptr[b + 1])])
+                          for b in range(wl.batch)])
+    flops, nbytes = algorithmic_work(inp, anc)
+    peaks, peak_kind = load_peaks()
+
+    attn = va.VerifyAttention(max_batch=wl.batch, num_heads=wl.num_heads, max_tree=max(wl.tree_sizes),
+                              max_kv_per_req=max(wl.kv_lens), max_total_kv=wl.total_kv, pool_slots=wl.pool_slots,
+                              sm_scale=wl.sm_scale)
+    d = wdev.to_device(inp, anc)
+    vargs = attn.make_args(*wdev.positional(d), lse=d["lse"], visible_count=d["visible_count"])
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    # Warm the kernels eagerly once, then capture split and reduce as two graphs.
+    with torch.cuda.stream(stream):
+        attn.run(vargs, stream.cuda_stream)
+        attn.reduce(vargs, stream.cuda_stream)
+    stream.synchronize()
+    g_run, g_red = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_run, stream=stream):
+        attn.run(vargs, stream.cuda_stream)
+    with torch.cuda.graph(g_red, stream=stream):
+        attn.reduce(vargs, stream.cuda_stream)
+    code, bits = attn.status(stream.cuda_stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits:#x}) after warm-up")
+
+    def step(ev):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            if ev is not None:
+                ev[0].record(stream)
+            g_run.replay()
+            if ev is not None:
+                ev[1].record(stream)
+            g_red.replay()
+            if ev is not None:
+                ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step(None)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = int(visible.split(",")[local_rank]) if visible and visible.split(",")[0].isdigit() else local_rank
+    with ClockSampler(gpu_index) as clocks:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            step(events[i])
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    clock_info = clocks.summary()
+    code, bits = attn.status(stream.cuda_stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits:#x}) after timing")
+    call_ms = [e[0].elapsed_time(e[2]) for e in events]
+    split_ms = [e[0].elapsed_time(e[1]) for e in events]
+    t_call = statistics.mean(call_ms) * 1e-3
+    t_split = statistics.mean(split_ms) * 1e-3
+
+    # End to end through the public call with host buffers: per step, copy
+    # this call's inputs (queries, slot list, indptrs, tree masks) from pinned
+    # host memory, run, and read the output and LSE back. The latent KV pool
+    # is the device-resident KV cache and is not copied.
+    host = {k: d[k].cpu().pin_memory() for k in ("q_latent", "q_rope", "kv_indices", "kv_indptr", "qo_indptr",
+                                                   "tree_anc")}
+    out_h = torch.empty_like(d["out"], device="cpu").pin_memory()
+    lse_h = torch.empty_like(d["lse"], device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    e2e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k, t in host.items():
+                d[k].copy_(t, non_blocking=True)
+            attn(*wdev.positional(d), lse=d["lse"], visible_count=d["visible_count"], stream=stream.cuda_stream)
+            out_h.copy_(d["out"], non_blocking=True)
+            lse_h.copy_(d["lse"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
+
+    if dist is not None:
+        t = torch.tensor([t_call, t_split, t_e2e], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_call, t_split, t_e2e = (float(x) for x in t.tolist())
+
+    kv = wl.total_kv
+    tflops_split = flops / t_split / 1e12
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    traffic_path = os.path.join(ROOT, "profiles", "split_kernel_long_traffic.json")
+    traffic = None
+    if os.path.exists(traffic_path):
+        with open(traffic_path) as f:
+            tr = json.load(f)
+        if tr.get("kernel_source_digest") == kernel_digest():
+            traffic = tr.get("dram_bytes_per_launch")
+
+    result = {
+        "metric": METRIC, "value": kv * world / t_call, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, {"parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
+                                       "graph": "split and reduce replayed from CUDA graphs"}),
+        "detail": {
+            "us_per_call": t_call * 1e6, "split_us": t_split * 1e6, "reduce_us": (t_call - t_split) * 1e6,
+            "kv_tok_per_s_per_gpu": kv / t_call,
+            "hbm_gbs_algorithmic": nbytes / t_call / 1e9,
+            "tflops_split": tflops_split,
+            "roofline_us": t_roof * 1e6, "roofline_frac_call": t_roof / t_call,
+            "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+            "peaks": {k: v for k, v in peaks.items()}, "peaks_kind": peak_kind,
+        },
+        "roofline": {"bound": "tensor", "achieved": tflops_split, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tflops_split / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_kind": f"{peak_kind} burst bf16 (cuBLAS), kernel timed alone"},
+        "clocks": clock_info,
+        "e2e": {"value": kv * world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+
+        result["cpu_baseline"] = cpu_baseline(inp, oracle.ancestor_masks(inp.parents, inp.qo_indptr))
+    if dist is not None:
+        dist.barrier()
+        del g_run, g_red
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def kernel_digest() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_speculative_verify_absorb_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * verify_attn.h -- C ABI of the B200 (sm_100a) MLA-absorb tree-verify attention.
+ *
+ * The operation ("MLA-absorb attention with a custom tree mask": page "The
+ * Execution Phase: From Plan to 3-6x Decode Speedup on Blackwell Consumer
+ * GPUs", section "The Transition: From Planning to Execution", item 3):
+ *
+ *   For request b with T_b tree nodes and a prefix of L_b tokens, its KV
+ *   sequence has N_b = L_b + T_b positions: the prefix in order, then the tree
+ *   nodes in node order (tree node i is position L_b + i). Position j lives
+ *   in pool row kv_pool[kv_indices[kv_indptr[b] + j]] (a page_size=1 pool:
+ *   page "The Verify Kernel Breakthrough", section "The Message in Context").
+ *   Every head of every tree node t attends
+ *     - every prefix position j < L_b, and
+ *     - tree position L_b + i iff bit i of tree_anc[qo_indptr[b] + t] is set
+ *       (ancestor-or-self mask; page "The Architecture Detective", section
+ *       "The Split Verify Design": dense prefix, masked tree block),
+ *   with scores  s_j = sm_scale * (q_latent[t,h,:] . c_kv[j,:] + q_rope[t,h,:] . k_rope[j,:])
+ *   and values c_kv[j, 0:512] (one latent row per token serves all heads:
+ *   page "The Execution Phase", section "The Core Design"), and writes
+ *     out[t,h,:] = softmax_j(s_j) . c_kv,   lse[t,h] = ln sum_j exp(s_j).
+ *
+ * Work split (page "The Verify Kernel Breakthrough", section "The Message in
+ * Context": KV-split flash-decode with partial+reduce): verify_attn_run
+ * writes fp32 partial states (m, l, O) per KV split into the caller's
+ * workspace; verify_attn_reduce merges them (LSE merge) into out/lse.
+ *
+ * Capture safety (page "The Execution Phase", section "Making the Kernel
+ * CUDA Graph Capture-Safe"): the library never allocates, never
+ * synchronises and never reads device data on the host inside run/reduce.
+ * The launch shape depends only on the plan, so a call can be captured into
+ * a CUDA graph and replayed while the per-request lengths in the device
+ * indptr arrays change, as long as they stay within the plan's maxima.
+ *
+ * Conventions for every function below:
+ *   - Pointers are DEVICE pointers unless the name ends in _h (host).
+ *   - The caller owns all memory; the library keeps no pointer after return.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Strides are in elements. Every bf16 row (one token and head of q, one
+ *     pool slot, one output row) must start on a 16-byte boundary: base
+ *     pointers 16-byte aligned, strides multiples of 8 elements.
+ *   - Return 0 on success or a negative VERIFY_ATTN_E* code; nothing is
+ *     launched when an argument check fails.
+ */
+#ifndef VERIFY_ATTN_H
+#define VERIFY_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *verify_attn_stream_t;
+
+#define VERIFY_ATTN_OK 0
+#define VERIFY_ATTN_EINVAL (-1)               /* bad pointer, size, stride, alignment or tree */
+#define VERIFY_ATTN_UNSUPPORTED (-2)          /* d_latent != 512, d_rope != 64, tree > 64 nodes, too many heads */
+#define VERIFY_ATTN_WORKSPACE_TOO_SMALL (-3)  /* ws_bytes below what the plan needs */
+#define VERIFY_ATTN_CUDA_ERROR (-4)           /* a CUDA launch or runtime call failed */
+#define VERIFY_ATTN_DEVICE_TIMEOUT (-5)       /* a bounded device-side wait gave up */
+#define VERIFY_ATTN_DEVICE_BAD_INPUT (-6)     /* device lengths/slots outside the plan; the bad part was skipped */
+
+#define VERIFY_ATTN_D_LATENT 512
+#define VERIFY_ATTN_D_ROPE 64
+#define VERIFY_ATTN_MAX_TREE 64
+#define VERIFY_ATTN_MAX_HEADS 1024
+#define VERIFY_ATTN_PLAN_VERSION 1
+
+/* Problem maxima a plan is made for (host struct, copied into the plan). */
+typedef struct {
+    int32_t max_batch;       /* >= 1: most requests per call */
+    int32_t num_heads;       /* H, 1..VERIFY_ATTN_MAX_HEADS */
+    int32_t max_tree;        /* most tree nodes per request, 1..64 */
+    int32_t d_latent;        /* must be 512 */
+    int32_t d_rope;          /* must be 64 */
+    int32_t num_sms;         /* SMs to plan for; 0 = ask the current device */
+    int64_t max_kv_per_req;  /* most KV positions (prefix + tree) per request, >= max_tree */
+    int64_t max_total_kv;    /* most KV positions summed over a call's requests */
+    int64_t pool_slots;      /* rows in kv_pool; every kv_indices entry must be below this */
+    float sm_scale;          /* softmax scale applied to the 576-wide dot product, finite and > 0 */
+    int32_t reserved;
+} verify_attn_params;
+
+/* Launch plan: plain data, filled by verify_attn_plan, read by run/reduce.
+ * Callers may copy it but should not edit it. */
+typedef struct {
+    int32_t version;            /* VERIFY_ATTN_PLAN_VERSION */
+    int32_t num_heads;
+    int32_t max_batch;
+    int32_t max_tree;
+    int64_t max_kv_per_req;
+    int64_t max_total_kv;
+    int64_t pool_slots;
+    float sm_scale;
+    int32_t num_clusters;       /* persistent CTA pairs of the split kernel */
+    int32_t rows_per_tile;      /* (token, head) query rows per CTA pair: 128 */
+    int32_t keys_per_tile;      /* KV positions per work unit: 128 */
+    int32_t row_tiles_per_req;  /* ceil(max_tree * num_heads / rows_per_tile) */
+    int32_t num_slots;          /* partial-state slots in the workspace */
+    int64_t ws_meta_offset;     /* bytes: float4 {m, l, count, 0} per slot row */
+    int64_t ws_partial_offset;  /* bytes: fp32 O[512] per slot row */
+    int64_t ws_bytes;           /* total workspace bytes */
+    int32_t split_smem_bytes;   /* dynamic shared memory of the split kernel */
+    int32_t reserved[7];
+} verify_attn_plan_t;
+
+/* Per-call arguments (device pointers). */
+typedef struct {
+    const uint16_t *q_latent;   /* bf16 [sumT, H, 512] */
+    int64_t q_latent_stride_tok, q_latent_stride_head;
+    const uint16_t *q_rope;     /* bf16 [sumT, H, 64] */
+    int64_t q_rope_stride_tok, q_rope_stride_head;
+    const uint16_t *kv_pool;    /* bf16 [pool_slots, >=576]: c_kv in 0..511, k_rope in 512..575 */
+    int64_t kv_row_stride;
+    const int32_t *kv_indices;  /* [sum N_b] pool slots: prefix positions, then tree nodes */
+    const int32_t *kv_indptr;   /* [batch+1] offsets into kv_indices; N_b = diff */
+    const int32_t *qo_indptr;   /* [batch+1] offsets into tokens; T_b = diff, 1..max_tree */
+    const uint64_t *tree_anc;   /* [sumT] ancestor-or-self bitmask over the request's tree nodes */
+    int32_t batch;              /* 1..max_batch (host value, fixed for a captured graph) */
+    int32_t reserved0;
+    uint16_t *out;              /* bf16 [sumT, H, 512] */
+    int64_t out_stride_tok, out_stride_head;
+    float *lse;                 /* [sumT, H] natural-log LSE, or NULL */
+    int32_t *visible_count;     /* [sumT] keys each node attended, or NULL */
+} verify_attn_args;
+
+/*
+ * Validate the maxima and fill *plan and *ws_bytes (host only; queries the
+ * current device's SM count when params->num_sms is 0, nothing else).
+ * Returns VERIFY_ATTN_EINVAL / VERIFY_ATTN_UNSUPPORTED on bad maxima.
+ */
+int verify_attn_plan(const verify_attn_params *params, verify_attn_plan_t *plan, size_t *ws_bytes);
+
+/*
+ * Zero the workspace's device status word (cudaMemsetAsync on `stream`).
+ * Call once after allocating a workspace and after reading a non-zero status.
+ */
+int verify_attn_workspace_init(const verify_attn_plan_t *plan, void *ws, size_t ws_bytes,
+                               verify_attn_stream_t stream);
+
+/*
+ * Split kernel: every persistent CTA pair takes an equal share of the
+ * (query-row tile, KV tile) units of the call, runs both contractions on the
+ * tensor cores and writes one fp32 partial state (m, l, O) per (row tile,
+ * pair) into ws. Asynchronous on `stream`, capture-safe. Device-side length
+ * or slot errors set the status word and skip the offending work.
+ */
+int verify_attn_run(const verify_attn_plan_t *plan, const verify_attn_args *args, void *ws,
+                    size_t ws_bytes, verify_attn_stream_t stream);
+
+/*
+ * Reduce kernel: LSE-merges every row's partial states from ws into
+ * args->out (bf16, round to nearest even), args->lse (natural log) and
+ * args->visible_count. Must follow verify_attn_run on the same stream with
+ * the same plan, args and ws. Asynchronous, capture-safe.
+ */
+int verify_attn_reduce(const verify_attn_plan_t *plan, const verify_attn_args *args, void *ws,
+                       size_t ws_bytes, verify_attn_stream_t stream);
+
+/*
+ * Host helper: ancestor-or-self masks of one tree from its parent array
+ * (parents_h[0] == -1 is the root, 0 <= parents_h[i] < i otherwise). Bit j of
+ * anc_h[i] is set iff node j is node i or one of its ancestors. T in 1..64.
+ * Returns VERIFY_ATTN_EINVAL for a malformed tree (anc_h untouched then).
+ */
+int verify_attn_build_tree_mask(const int32_t *parents_h, int32_t T, uint64_t *anc_h);
+
+/*
+ * Read the workspace's device status word: copies it to the host on
+ * `stream` and synchronises that stream (not capture-safe; call after the
+ * work you want to check). Returns VERIFY_ATTN_OK, VERIFY_ATTN_DEVICE_TIMEOUT,
+ * VERIFY_ATTN_DEVICE_BAD_INPUT or VERIFY_ATTN_CUDA_ERROR; *detail_h (may be
+ * NULL) receives the raw status bits.
+ */
+int verify_attn_status(const void *ws, verify_attn_stream_t stream, uint32_t *detail_h);
+
+/* Static string for a return code. */
+const char *verify_attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VERIFY_ATTN_H */
