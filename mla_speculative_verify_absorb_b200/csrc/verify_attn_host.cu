@@ -60,7 +60,7 @@ int verify_attn_plan(const verify_attn_params* params, verify_attn_plan_t* plan,
   if (q.max_tree > VERIFY_ATTN_MAX_TREE || q.num_heads > VERIFY_ATTN_MAX_HEADS) return VERIFY_ATTN_UNSUPPORTED;
   if (q.max_kv_per_req < q.max_tree || q.max_kv_per_req > INT32_MAX) return VERIFY_ATTN_EINVAL;
   if (q.max_total_kv < q.max_tree || q.max_total_kv > INT32_MAX) return VERIFY_ATTN_EINVAL;
-  if (q.pool_slots < 1 || q.pool_slots > (int64_t)INT32_MAX + 1) return VERIFY_ATTN_EINVAL;
+  if (q.pool_slots < 1 || q.pool_slots > INT32_MAX) return VERIFY_ATTN_EINVAL;
   if (!(q.sm_scale > 0.f) || !isfinite(q.sm_scale)) return VERIFY_ATTN_EINVAL;
 
   // Persistent CTA pairs: half the SMs, or fewer if the device cannot keep

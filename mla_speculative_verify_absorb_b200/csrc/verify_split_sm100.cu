@@ -34,6 +34,7 @@
 //    request lengths, and at most G + #row tiles partial states are written.
 //  * Every wait is bounded; on expiry the kernel records it in the status
 //    word, unwinds both CTAs and frees its tensor memory.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -47,14 +48,14 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 224;          // 4 softmax + 2 producer + 1 MMA warps
+constexpr int kThreads = 224;          // 4 softmax + KV producer + Q loader + MMA warps
 constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerWarp0 = 4;
+constexpr int kKvWarp = 4;
+constexpr int kQWarp = 5;
 constexpr int kMmaWarp = 6;
 
 constexpr int kStageBytes = 8192;
-constexpr int kNumStages = 12;
-constexpr int kPendingStages = 4;      // cp.async groups a producer keeps in flight
+constexpr int kNumStages = 14;
 constexpr int kQBlocks = kDQK / 64;    // 9 chunks of 64 columns
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQBlocks * 8192;   // 2 buffers x 2 key blocks x 8 KB
@@ -206,122 +207,87 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// ----------------------------------------------------------------------------- producer
+// ----------------------------------------------------------------------------- producers
 
-struct Producer {
+// Warp 4: streams the K and V stages of every tile with TMA gathers. Lane l
+// holds the pool slots of the tile's keys 4l..4l+3 and issues the gather4s
+// that need them; slots are read one tile ahead. Each stage is 8 KB per CTA
+// and its bytes are counted on the leader CTA's ring_full barrier, which
+// also expects one arrival from each CTA's producer.
+struct KvProducer {
   const SplitParams& p;
+  const void* tmap;
   Ctrl* ctrl;
   uint8_t* smem;
-  uint32_t rank, leader_base;
-  int pt;                      // 0..63
-  uint32_t st = 0;             // global stage counter
-  uint32_t npending = 0;       // stages st-npending .. st-1 are copied but not yet announced
-  bool ok = true;
+  uint32_t rank;
+  int lane;
+  uint32_t st = 0;
 
-  __device__ Producer(const SplitParams& p_, Ctrl* c, uint8_t* s, uint32_t r, int t)
-      : p(p_), ctrl(c), smem(s), rank(r), pt(t) {}
-
-  __device__ uint32_t leader_bar(const uint64_t* bar) { return map_to_rank(smem_addr(bar), 0); }
-
-  __device__ void arrive_stage(uint32_t stage) {
-    fence_proxy_async_smem();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(leader_bar(&ctrl->ring_full[stage]));
+  __device__ KvProducer(const SplitParams& p_, const void* m, Ctrl* c, uint8_t* s, uint32_t r)
+      : p(p_), tmap(m), ctrl(c), smem(s), rank(r) {
+    lane = threadIdx.x & 31;
   }
 
-  __device__ void flush() {
-    cp_async_wait<0>();
-    for (uint32_t i = npending; i > 0; --i) arrive_stage((st - i) % kNumStages);
-    npending = 0;
+  // Pool slots of keys 4*lane .. 4*lane+3 of tile kt; positions past the
+  // request, or slots outside the pool, become an out-of-range row that the
+  // TMA fills with zeros.
+  __device__ void load_slots(const Segment& s, int64_t kt, int32_t (&sl)[4]) {
+    const int64_t pos0 = kt * kKeysPerTile + 4 * lane;
+    const int32_t oob = (int32_t)p.pool_slots;   // first row past the pool (pool_slots <= INT32_MAX)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t pos = pos0 + e;
+      int32_t v = oob;
+      if (pos < s.req.N) {
+        v = p.kv_indices[s.req.kv_begin + pos];
+        if (v < 0 || (int64_t)v >= p.pool_slots) {
+          atomicOr(p.status, kStatusBadSlot);
+          v = oob;
+        }
+      }
+      sl[e] = v;
+    }
   }
 
-  // Claim the next ring stage (waits until the MMA released its last use).
-  __device__ bool acquire(uint32_t& stage) {
+  // Claim the next ring stage and announce its bytes on the leader's barrier.
+  __device__ bool acquire(uint32_t& stage, uint32_t& bar) {
     stage = st % kNumStages;
-    uint32_t use = st / kNumStages;
+    const uint32_t use = st / kNumStages;
     if (use >= 1 && !wait_warp(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return false;
-    return true;
-  }
-
-  __device__ void commit() {
-    cp_async_commit();
-    ++npending;
-    ++st;
-    if (npending > kPendingStages) {
-      cp_async_wait<kPendingStages>();
-      arrive_stage((st - npending) % kNumStages);
-      --npending;
-    }
-  }
-
-  __device__ int32_t slot_of(const Segment& s, int64_t pos, bool& valid) {
-    valid = pos < s.req.N;
-    if (!valid) return 0;
-    int32_t slot = p.kv_indices[s.req.kv_begin + pos];
-    if (slot < 0 || (int64_t)slot >= p.pool_slots) {
-      atomicOr(p.status, kStatusBadSlot);
-      valid = false;
-      return 0;
-    }
-    return slot;
-  }
-
-  __device__ void load_q(const Segment& s) {
-    const int64_t rows = (int64_t)s.req.T * p.num_heads;
-    const int64_t gr = (int64_t)s.rt * kRowsPerTile + rank * kRowsPerCta + pt;
-    const bool valid = gr < rows;
-    const int64_t t = valid ? gr / p.num_heads : 0, h = valid ? gr % p.num_heads : 0;
-    const uint16_t* ql = p.q_latent + (s.req.q_begin + t) * p.ql_tok + h * p.ql_head;
-    const uint16_t* qr = p.q_rope + (s.req.q_begin + t) * p.qr_tok + h * p.qr_head;
-    const uint32_t base = smem_addr(smem + kOffQ) + pt * 128;
-    const uint32_t nbytes = valid ? 16u : 0u;
-#pragma unroll 8
-    for (int c = 0; c < 64; ++c)
-      cp_async_16(base + (c >> 3) * 8192 + (((c & 7) ^ (pt & 7)) << 4), ql + c * 8, nbytes);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) cp_async_16(base + 8 * 8192 + ((c ^ (pt & 7)) << 4), qr + c * 8, nbytes);
-    cp_async_commit();
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
+    bar = map_to_rank(smem_addr(&ctrl->ring_full[stage]), 0);
+    if (lane == 0) mbar_arrive_expect_tx_cluster(bar, kStageBytes);
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(leader_bar(&ctrl->q_full));
+    ++st;
+    return true;
   }
 
-  // Nine stages: this CTA's 64 keys of the tile, 64 score columns each.
-  __device__ bool load_k(const Segment& s, int i) {
-    const int64_t kt = s.kt0 + i;
-    bool valid;
-    const int32_t slot = slot_of(s, kt * kKeysPerTile + rank * 64 + pt, valid);
-    const uint16_t* row = p.kv_pool + (int64_t)slot * p.kv_stride;
-    const uint32_t nbytes = valid ? 16u : 0u;
+  // Nine stages: this CTA's 64 keys (lanes 16*rank .. 16*rank+15) x 64 score columns each.
+  __device__ bool load_k(const int32_t (&sl)[4]) {
+    const int first = 16 * (int)rank;
     for (int kb = 0; kb < kQBlocks; ++kb) {
-      uint32_t stage;
-      if (!acquire(stage)) return false;
-      const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + pt * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) cp_async_16(dst + ((c ^ (pt & 7)) << 4), row + kb * 64 + c * 8, nbytes);
-      commit();
+      uint32_t stage, bar;
+      if (!acquire(stage, bar)) return false;
+      if (lane >= first && lane < first + 16) {
+        const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + (lane - first) * 512;
+        tma_gather4_2sm(dst, tmap, kb * 64, sl[0], sl[1], sl[2], sl[3], bar);
+      }
     }
     return true;
   }
 
-  // Eight stages: 32 keys x this CTA's 128 value columns of one output half.
-  __device__ bool load_v(const Segment& s, int i) {
-    const int64_t kt = s.kt0 + i;
-    const int k = pt & 31, blk = pt >> 5;
+  // Eight stages: 32 keys (lanes 8*kc .. 8*kc+7) x this CTA's 128 value
+  // columns of one output half, as two 64-column blocks.
+  __device__ bool load_v(const int32_t (&sl)[4]) {
     for (int kc = 0; kc < 4; ++kc) {
-      bool valid;
-      const int32_t slot = slot_of(s, kt * kKeysPerTile + kc * 32 + k, valid);
-      const uint16_t* row = p.kv_pool + (int64_t)slot * p.kv_stride;
-      const uint32_t nbytes = valid ? 16u : 0u;
       for (int dh = 0; dh < 2; ++dh) {
-        uint32_t stage;
-        if (!acquire(stage)) return false;
-        const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + blk * 4096 + k * 128;
-        const uint16_t* src = row + dh * 256 + rank * 128 + blk * 64;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cp_async_16(dst + ((c ^ (k & 7)) << 4), src + c * 8, nbytes);
-        commit();
+        uint32_t stage, bar;
+        if (!acquire(stage, bar)) return false;
+        if (lane >= 8 * kc && lane < 8 * kc + 8) {
+          const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + (lane - 8 * kc) * 512;
+          const int32_t col = dh * 256 + (int32_t)rank * 128;
+          tma_gather4_2sm(dst, tmap, col, sl[0], sl[1], sl[2], sl[3], bar);
+          tma_gather4_2sm(dst + 4096, tmap, col + 64, sl[0], sl[1], sl[2], sl[3], bar);
+        }
       }
     }
     return true;
@@ -329,20 +295,67 @@ struct Producer {
 
   __device__ void run(int64_t u0, int64_t u1) {
     Segment s;
+    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
+      int32_t cur[4], prev[4], next[4];
+      load_slots(s, s.kt0, cur);
+      for (int i = 0; i < s.n; ++i) {
+        if (i + 1 < s.n) load_slots(s, s.kt0 + i + 1, next);
+        if (!load_k(cur)) return;
+        if (i >= 1 && !load_v(prev)) return;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          prev[e] = cur[e];
+          cur[e] = next[e];
+        }
+      }
+      if (!load_v(prev)) return;
+    }
+  }
+};
+
+// Warp 5: loads the CTA's 64 query rows of each segment's row tile into the
+// swizzled Q buffer with 16-byte cp.async (after the previous segment's last
+// score MMA released it), then announces them on the leader's q_full.
+struct QLoader {
+  const SplitParams& p;
+  Ctrl* ctrl;
+  uint8_t* smem;
+  uint32_t rank;
+  int lane;
+
+  __device__ QLoader(const SplitParams& p_, Ctrl* c, uint8_t* s, uint32_t r) : p(p_), ctrl(c), smem(s), rank(r) {
+    lane = threadIdx.x & 31;
+  }
+
+  __device__ void load_row(const Segment& s, int row) {
+    const int64_t rows = (int64_t)s.req.T * p.num_heads;
+    const int64_t gr = (int64_t)s.rt * kRowsPerTile + rank * kRowsPerCta + row;
+    const bool valid = gr < rows;
+    const int64_t t = valid ? gr / p.num_heads : 0, h = valid ? gr % p.num_heads : 0;
+    const uint16_t* ql = p.q_latent + (s.req.q_begin + t) * p.ql_tok + h * p.ql_head;
+    const uint16_t* qr = p.q_rope + (s.req.q_begin + t) * p.qr_tok + h * p.qr_head;
+    const uint32_t base = smem_addr(smem + kOffQ) + row * 128;
+    const uint32_t nbytes = valid ? 16u : 0u;
+#pragma unroll 8
+    for (int c = 0; c < 64; ++c)
+      cp_async_16(base + (c >> 3) * 8192 + (((c & 7) ^ (row & 7)) << 4), ql + c * 8, nbytes);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) cp_async_16(base + 8 * 8192 + ((c ^ (row & 7)) << 4), qr + c * 8, nbytes);
+  }
+
+  __device__ void run(int64_t u0, int64_t u1) {
+    Segment s;
     int si = 0;
     for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n, ++si) {
-      if (si > 0) {
-        flush();
-        if (!wait_warp(smem_addr(&ctrl->q_empty), (si - 1) & 1, ctrl, p, rank)) return;
-      }
-      load_q(s);
-      for (int i = 0; i < s.n; ++i) {
-        if (!load_k(s, i)) return;
-        if (i >= 1 && !load_v(s, i - 1)) return;
-      }
-      if (!load_v(s, s.n - 1)) return;
+      if (si > 0 && !wait_warp(smem_addr(&ctrl->q_empty), (si - 1) & 1, ctrl, p, rank)) return;
+      load_row(s, lane);
+      load_row(s, lane + 32);
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_addr(&ctrl->q_full), 0));
     }
-    flush();
   }
 };
 
@@ -601,7 +614,7 @@ struct Softmax {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    verify_split_kernel(const SplitParams p) {
+    verify_split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap kv_map) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kOffCtrl);
@@ -612,7 +625,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumStages; ++s) {
-      mbar_init(smem_addr(&ctrl->ring_full[s]), 4);   // 2 producer warps x 2 CTAs
+      mbar_init(smem_addr(&ctrl->ring_full[s]), 2);   // one KV producer per CTA (+ TMA bytes)
       mbar_init(smem_addr(&ctrl->ring_empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -620,7 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&ctrl->p_full[b]), 8);       // 4 softmax warps x 2 CTAs
       mbar_init(smem_addr(&ctrl->pv_done[b]), 1);
     }
-    mbar_init(smem_addr(&ctrl->q_full), 4);
+    mbar_init(smem_addr(&ctrl->q_full), 2);         // one Q loader warp per CTA
     mbar_init(smem_addr(&ctrl->q_empty), 1);
     mbar_init(smem_addr(&ctrl->o_free), 8);
     mbar_init(smem_addr(&ctrl->mma_final), 1);
@@ -632,6 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_alloc_2sm(smem_addr(&ctrl->tmem_base), kTmemCols);
     tmem_relinquish_2sm();
   }
+  if (warp == kKvWarp && (threadIdx.x & 31) == 0) prefetch_tmap(&kv_map);
   tc_fence_before();
   __syncthreads();
   cluster_sync();
@@ -645,9 +659,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
-  } else if (warp < kMmaWarp) {
-    Producer pr(p, ctrl, smem, rank, (int)threadIdx.x - kProducerWarp0 * 32);
+  } else if (warp == kKvWarp) {
+    KvProducer pr(p, &kv_map, ctrl, smem, rank);
     pr.run(u0, u1);
+  } else if (warp == kQWarp) {
+    QLoader ql(p, ctrl, smem, rank);
+    ql.run(u0, u1);
     cp_async_wait<0>();
   } else if (rank == 0) {
     if ((threadIdx.x & 31) == 0) {
@@ -699,10 +716,39 @@ cudaError_t split_max_active_clusters(int* n) {
   return cudaOccupancyMaxActiveClusters(n, verify_split_kernel, &cfg);
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Tensor map over the latent pool: [pool_slots rows, 576 bf16 columns], row
+// stride from the caller, boxes of 64 columns x 1 row, 128-byte swizzle (the
+// layout the tensor-core operands expect), zeros for rows outside the pool.
+static cudaError_t encode_pool_map(const SplitParams& p, CUtensorMap* map) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)kDQK, (cuuint64_t)p.pool_slots};
+  const cuuint64_t strides[1] = {(cuuint64_t)p.kv_stride * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estride[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.kv_pool), dims, strides, box,
+                      estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream) {
   cudaError_t e = configure_split();
   if (e != cudaSuccess) return e;
-  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p);
+  CUtensorMap map;
+  e = encode_pool_map(p, &map);
+  if (e != cudaSuccess) return e;
+  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, map);
   return cudaGetLastError();
 }
 
