@@ -106,6 +106,12 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
+// Arrive on a local barrier once all of this thread's earlier cp.async copies
+// have landed (the arrival is made by the hardware; the thread does not wait).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");

@@ -34,7 +34,6 @@
 //    request lengths, and at most G + #row tiles partial states are written.
 //  * Every wait is bounded; on expiry the kernel records it in the status
 //    word, unwinds both CTAs and frees its tensor memory.
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -48,11 +47,13 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 224;          // 4 softmax + KV producer + Q loader + MMA warps
+constexpr int kThreads = 352;          // 4 softmax + 4 KV loader + Q loader + relay + MMA warps
 constexpr int kSoftmaxThreads = 128;
-constexpr int kKvWarp = 4;
-constexpr int kQWarp = 5;
-constexpr int kMmaWarp = 6;
+constexpr int kKvWarp0 = 4;
+constexpr int kNumKvWarps = 4;
+constexpr int kQWarp = 8;
+constexpr int kRelayWarp = 9;
+constexpr int kMmaWarp = 10;
 
 constexpr int kStageBytes = 8192;
 constexpr int kNumStages = 14;
@@ -74,7 +75,8 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct Ctrl {
-  uint64_t ring_full[kNumStages];
+  uint64_t ring_full[kNumStages];   // leader: 32 loader-lane arrivals + 1 relay arrival per stage
+  uint64_t peer_full[kNumStages];   // peer: 32 loader-lane arrivals, relayed to the leader
   uint64_t ring_empty[kNumStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
@@ -209,106 +211,179 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ----------------------------------------------------------------------------- producers
 
-// Warp 4: streams the K and V stages of every tile with TMA gathers. Lane l
-// holds the pool slots of the tile's keys 4l..4l+3 and issues the gather4s
-// that need them; slots are read one tile ahead. Each stage is 8 KB per CTA
-// and its bytes are counted on the leader CTA's ring_full barrier, which
-// also expects one arrival from each CTA's producer.
-struct KvProducer {
+// Stage order of one segment of n tiles, shared by the loaders, the relay and
+// the MMA issuer: K(0), then for i = 1..n-1: K(i), V(i-1), then V(n-1). K(i)
+// is 9 stages (64-column blocks of the 576 score columns), V(i) 8 stages
+// (4 key chunks of 32 x 2 output halves), so a segment has 17n stages.
+constexpr int kStagesK = kQBlocks;    // 9
+constexpr int kStagesV = 8;
+constexpr int kStagesPerTile = kStagesK + kStagesV;
+
+struct StageDesc {
+  int32_t tile;    // tile index within the segment
+  int32_t is_v;    // 0: K stage, 1: V stage
+  int32_t idx;     // K: column block 0..8; V: kc*2 + dh
+};
+
+__device__ __forceinline__ StageDesc describe_stage(uint32_t p, int n) {
+  StageDesc d;
+  if (p < (uint32_t)kStagesK) {
+    d.tile = 0; d.is_v = 0; d.idx = (int)p;
+    return d;
+  }
+  const uint32_t q = p - kStagesK;
+  const uint32_t blk = q / kStagesPerTile, r = q % kStagesPerTile;
+  if (blk < (uint32_t)(n - 1)) {
+    if (r < (uint32_t)kStagesK) { d.tile = (int)blk + 1; d.is_v = 0; d.idx = (int)r; }
+    else { d.tile = (int)blk; d.is_v = 1; d.idx = (int)r - kStagesK; }
+  } else {
+    d.tile = n - 1; d.is_v = 1; d.idx = (int)(q - (uint32_t)(n - 1) * kStagesPerTile);
+  }
+  return d;
+}
+
+// Walks the cluster's segments forward to find the segment of stage st.
+struct StageCursor {
   const SplitParams& p;
-  const void* tmap;
+  int64_t u, u1;
+  Segment seg;
+  uint32_t base = 0;   // first global stage of seg
+  bool valid = false;
+
+  __device__ StageCursor(const SplitParams& p_, int64_t u0, int64_t u1_) : p(p_), u(u0), u1(u1_) {
+    valid = find_segment(p, u, u1, seg);
+  }
+  // Position seg so that base <= st < base + 17 n; false once past the end.
+  __device__ bool seek(uint32_t st) {
+    while (valid && st >= base + (uint32_t)kStagesPerTile * seg.n) {
+      base += (uint32_t)kStagesPerTile * seg.n;
+      u += seg.n;
+      valid = find_segment(p, u, u1, seg);
+    }
+    return valid;
+  }
+};
+
+// Warps 4-7: gather the K and V stages of every tile with 16-byte cp.async.
+// Loader warp w fills global stages w, w+4, w+8, ...; each lane copies 16
+// chunks of 16 bytes (4 keys x 128 B per warp instruction) into the
+// 128-byte-swizzled stage and the hardware arrives on the CTA-local full
+// barrier once they land (leader: ring_full, peer: peer_full, relayed). The
+// pool slots of the warp's next stage are fetched while the current stage is
+// issued. Rows past the request or with a slot outside the pool are zero.
+struct KvLoader {
+  const SplitParams& p;
   Ctrl* ctrl;
   uint8_t* smem;
   uint32_t rank;
-  int lane;
-  uint32_t st = 0;
+  int warp, lane;
 
-  __device__ KvProducer(const SplitParams& p_, const void* m, Ctrl* c, uint8_t* s, uint32_t r)
-      : p(p_), tmap(m), ctrl(c), smem(s), rank(r) {
+  __device__ KvLoader(const SplitParams& p_, Ctrl* c, uint8_t* s, uint32_t r, int w)
+      : p(p_), ctrl(c), smem(s), rank(r), warp(w) {
     lane = threadIdx.x & 31;
   }
 
-  // Pool slots of keys 4*lane .. 4*lane+3 of tile kt; positions past the
-  // request, or slots outside the pool, become an out-of-range row that the
-  // TMA fills with zeros.
-  __device__ void load_slots(const Segment& s, int64_t kt, int32_t (&sl)[4]) {
-    const int64_t pos0 = kt * kKeysPerTile + 4 * lane;
-    const int32_t oob = (int32_t)p.pool_slots;   // first row past the pool (pool_slots <= INT32_MAX)
+  // Position (within the request) of the key this lane copies in chunk group j.
+  __device__ __forceinline__ int64_t key_pos(const Segment& s, const StageDesc& d, int j) const {
+    const int64_t kt = s.kt0 + d.tile;
+    if (!d.is_v) return kt * kKeysPerTile + rank * 64 + j * 4 + (lane >> 3);
+    const int kc = d.idx >> 1;
+    return kt * kKeysPerTile + kc * 32 + (j & 7) * 4 + (lane >> 3);
+  }
+
+  __device__ __forceinline__ void load_slots(const Segment& s, const StageDesc& d, int32_t (&sl)[16]) {
+    const int nkeys = d.is_v ? 8 : 16;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int64_t pos = pos0 + e;
-      int32_t v = oob;
+    for (int j = 0; j < 16; ++j) {
+      if (j >= nkeys) break;
+      const int64_t pos = key_pos(s, d, j);
+      int32_t v = -1;
       if (pos < s.req.N) {
         v = p.kv_indices[s.req.kv_begin + pos];
         if (v < 0 || (int64_t)v >= p.pool_slots) {
           atomicOr(p.status, kStatusBadSlot);
-          v = oob;
+          v = -1;
         }
       }
-      sl[e] = v;
+      sl[j] = v;
     }
   }
 
-  // Claim the next ring stage and announce its bytes on the leader's barrier.
-  __device__ bool acquire(uint32_t& stage, uint32_t& bar) {
-    stage = st % kNumStages;
-    const uint32_t use = st / kNumStages;
-    if (use >= 1 && !wait_warp(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return false;
-    bar = map_to_rank(smem_addr(&ctrl->ring_full[stage]), 0);
-    if (lane == 0) mbar_arrive_expect_tx_cluster(bar, kStageBytes);
-    __syncwarp();
-    ++st;
-    return true;
-  }
-
-  // Nine stages: this CTA's 64 keys (lanes 16*rank .. 16*rank+15) x 64 score columns each.
-  __device__ bool load_k(const int32_t (&sl)[4]) {
-    const int first = 16 * (int)rank;
-    for (int kb = 0; kb < kQBlocks; ++kb) {
-      uint32_t stage, bar;
-      if (!acquire(stage, bar)) return false;
-      if (lane >= first && lane < first + 16) {
-        const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + (lane - first) * 512;
-        tma_gather4_2sm(dst, tmap, kb * 64, sl[0], sl[1], sl[2], sl[3], bar);
+  __device__ __forceinline__ void issue(const StageDesc& d, const int32_t (&sl)[16], uint32_t stage) {
+    const uint32_t base = smem_addr(smem + kOffRing + stage * kStageBytes);
+    const int ch = lane & 7;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      int key, col, slot_j;
+      uint32_t dst;
+      if (!d.is_v) {
+        key = j * 4 + (lane >> 3);
+        slot_j = sl[j];
+        col = d.idx * 64 + ch * 8;
+        dst = base + key * 128 + ((ch ^ (key & 7)) << 4);
+      } else {
+        const int blk = j >> 3, dh = d.idx & 1;
+        key = (j & 7) * 4 + (lane >> 3);
+        slot_j = sl[j & 7];
+        col = dh * 256 + (int)rank * 128 + blk * 64 + ch * 8;
+        dst = base + blk * 4096 + key * 128 + ((ch ^ (key & 7)) << 4);
       }
+      const bool ok = slot_j >= 0;
+      const uint16_t* src = p.kv_pool + (ok ? (int64_t)slot_j * p.kv_stride + col : 0);
+      cp_async_16(dst, src, ok ? 16u : 0u);
     }
-    return true;
-  }
-
-  // Eight stages: 32 keys (lanes 8*kc .. 8*kc+7) x this CTA's 128 value
-  // columns of one output half, as two 64-column blocks.
-  __device__ bool load_v(const int32_t (&sl)[4]) {
-    for (int kc = 0; kc < 4; ++kc) {
-      for (int dh = 0; dh < 2; ++dh) {
-        uint32_t stage, bar;
-        if (!acquire(stage, bar)) return false;
-        if (lane >= 8 * kc && lane < 8 * kc + 8) {
-          const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes) + (lane - 8 * kc) * 512;
-          const int32_t col = dh * 256 + (int32_t)rank * 128;
-          tma_gather4_2sm(dst, tmap, col, sl[0], sl[1], sl[2], sl[3], bar);
-          tma_gather4_2sm(dst + 4096, tmap, col + 64, sl[0], sl[1], sl[2], sl[3], bar);
-        }
-      }
-    }
-    return true;
   }
 
   __device__ void run(int64_t u0, int64_t u1) {
-    Segment s;
-    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
-      int32_t cur[4], prev[4], next[4];
-      load_slots(s, s.kt0, cur);
-      for (int i = 0; i < s.n; ++i) {
-        if (i + 1 < s.n) load_slots(s, s.kt0 + i + 1, next);
-        if (!load_k(cur)) return;
-        if (i >= 1 && !load_v(prev)) return;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          prev[e] = cur[e];
-          cur[e] = next[e];
-        }
+    StageCursor cur(p, u0, u1), nxt(p, u0, u1);
+    uint32_t st = (uint32_t)warp;
+    if (!cur.seek(st)) return;
+    StageDesc d = describe_stage(st - cur.base, cur.seg.n);
+    int32_t sl[16], sl_next[16];
+    load_slots(cur.seg, d, sl);
+    uint64_t* local_full = rank == 0 ? ctrl->ring_full : ctrl->peer_full;
+    while (true) {
+      const uint32_t st_next = st + kNumKvWarps;
+      const bool has_next = nxt.seek(st_next);
+      StageDesc dn;
+      if (has_next) {
+        dn = describe_stage(st_next - nxt.base, nxt.seg.n);
+        load_slots(nxt.seg, dn, sl_next);
       }
-      if (!load_v(prev)) return;
+      const uint32_t stage = st % kNumStages, use = st / kNumStages;
+      if (use >= 1 && !wait_warp(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return;
+      issue(d, sl, stage);
+      cp_async_arrive_noinc(smem_addr(&local_full[stage]));
+      if (!has_next) return;
+      st = st_next;
+      d = dn;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sl[j] = sl_next[j];
+    }
+  }
+};
+
+// Warp 9 of the peer CTA: forwards the completion of each of its stages to the
+// leader's ring_full after making the cp.async-written bytes visible to the
+// tensor core (async proxy).
+struct Relay {
+  const SplitParams& p;
+  Ctrl* ctrl;
+  uint32_t rank;
+
+  __device__ Relay(const SplitParams& p_, Ctrl* c, uint32_t r) : p(p_), ctrl(c), rank(r) {}
+
+  __device__ void run(int64_t u0, int64_t u1) {
+    Segment s;
+    uint32_t st = 0;
+    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
+      const uint32_t end = st + (uint32_t)kStagesPerTile * s.n;
+      for (; st < end; ++st) {
+        const uint32_t stage = st % kNumStages;
+        if (!wait_one(smem_addr(&ctrl->peer_full[stage]), (st / kNumStages) & 1u, ctrl, p, rank)) return;
+        fence_proxy_async_smem();
+        mbar_arrive_cluster(map_to_rank(smem_addr(&ctrl->ring_full[stage]), 0));
+      }
     }
   }
 };
@@ -384,6 +459,7 @@ struct Issuer {
     for (int kb = 0; kb < kQBlocks; ++kb) {
       const uint32_t stage = st % kNumStages;
       if (!wait_bar(&ctrl->ring_full[stage], (st / kNumStages) & 1u)) return false;
+      fence_proxy_async_smem();
       const uint32_t b0 = smem_addr(smem + kOffRing + stage * kStageBytes);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -403,6 +479,7 @@ struct Issuer {
       for (int dh = 0; dh < 2; ++dh) {
         const uint32_t stage = st % kNumStages;
         if (!wait_bar(&ctrl->ring_full[stage], (st / kNumStages) & 1u)) return false;
+        fence_proxy_async_smem();
         const uint32_t b0 = smem_addr(smem + kOffRing + stage * kStageBytes);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
@@ -614,7 +691,7 @@ struct Softmax {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    verify_split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap kv_map) {
+    verify_split_kernel(const SplitParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kOffCtrl);
@@ -625,7 +702,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumStages; ++s) {
-      mbar_init(smem_addr(&ctrl->ring_full[s]), 2);   // one KV producer per CTA (+ TMA bytes)
+      mbar_init(smem_addr(&ctrl->ring_full[s]), 32 + 1);   // the stage's loader warp lanes + the peer's relay
+      mbar_init(smem_addr(&ctrl->peer_full[s]), 32);       // the peer's loader warp lanes
       mbar_init(smem_addr(&ctrl->ring_empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -645,7 +723,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_alloc_2sm(smem_addr(&ctrl->tmem_base), kTmemCols);
     tmem_relinquish_2sm();
   }
-  if (warp == kKvWarp && (threadIdx.x & 31) == 0) prefetch_tmap(&kv_map);
   tc_fence_before();
   __syncthreads();
   cluster_sync();
@@ -659,9 +736,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
-  } else if (warp == kKvWarp) {
-    KvProducer pr(p, &kv_map, ctrl, smem, rank);
-    pr.run(u0, u1);
+  } else if (warp >= kKvWarp0 && warp < kKvWarp0 + kNumKvWarps) {
+    KvLoader ld(p, ctrl, smem, rank, warp - kKvWarp0);
+    ld.run(u0, u1);
+    cp_async_wait<0>();
+  } else if (warp == kRelayWarp) {
+    if (rank == 1 && (threadIdx.x & 31) == 0) {
+      Relay rl(p, ctrl, rank);
+      rl.run(u0, u1);
+    }
+    __syncwarp();
   } else if (warp == kQWarp) {
     QLoader ql(p, ctrl, smem, rank);
     ql.run(u0, u1);
@@ -716,39 +800,10 @@ cudaError_t split_max_active_clusters(int* n) {
   return cudaOccupancyMaxActiveClusters(n, verify_split_kernel, &cfg);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// Tensor map over the latent pool: [pool_slots rows, 576 bf16 columns], row
-// stride from the caller, boxes of 64 columns x 1 row, 128-byte swizzle (the
-// layout the tensor-core operands expect), zeros for rows outside the pool.
-static cudaError_t encode_pool_map(const SplitParams& p, CUtensorMap* map) {
-  static EncodeTiledFn encode = nullptr;
-  if (!encode) {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
-    encode = reinterpret_cast<EncodeTiledFn>(fn);
-  }
-  const cuuint64_t dims[2] = {(cuuint64_t)kDQK, (cuuint64_t)p.pool_slots};
-  const cuuint64_t strides[1] = {(cuuint64_t)p.kv_stride * 2};
-  const cuuint32_t box[2] = {64, 1};
-  const cuuint32_t estride[2] = {1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.kv_pool), dims, strides, box,
-                      estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream) {
   cudaError_t e = configure_split();
   if (e != cudaSuccess) return e;
-  CUtensorMap map;
-  e = encode_pool_map(p, &map);
-  if (e != cudaSuccess) return e;
-  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, map);
+  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
