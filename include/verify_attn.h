@@ -180,6 +180,38 @@ int verify_attn_status(const void *ws, verify_attn_stream_t stream, uint32_t *de
 /* Static string for a return code. */
 const char *verify_attn_strerror(int code);
 
+/* Size of the library-owned workspace used by verify_attn_forward_static. */
+#define VERIFY_ATTN_STATIC_WS_BYTES (32u << 20)
+
+/*
+ * verify_attn_forward_static -- run + reduce without any allocation.
+ *
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory when they run the verify step: a serving loop
+ * that must stay allocation-free after warm-up, a runtime that owns the device
+ * heap and forbids other allocators, or a plugin that only receives the
+ * tensors it may read and write. Such a caller passes its inputs and outputs
+ * as for verify_attn_run / verify_attn_reduce; the scratch those kernels need
+ * comes from a fixed array of VERIFY_ATTN_STATIC_WS_BYTES (32 MiB) inside the
+ * library, which every GPU that uses the library keeps until the process
+ * exits.
+ *
+ * - Plans whose ws_bytes exceed VERIFY_ATTN_STATIC_WS_BYTES are rejected with
+ *   VERIFY_ATTN_WORKSPACE_TOO_SMALL before anything is launched.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture on the device.
+ * - Every call shares the one array, which keeps the previous call's
+ *   contents; the call clears the status word itself. Calls that overlap on
+ *   the GPU (other streams, other host threads) race on it.
+ * - status: a caller-owned device uint32 that receives the status word at
+ *   the end of the call (same bits as verify_attn_status), or NULL.
+ * - No cudaMalloc, cudaFree or other allocating routine is called.
+ * Returns the same codes as verify_attn_run / verify_attn_reduce.
+ */
+int verify_attn_forward_static(const verify_attn_plan_t *plan, const verify_attn_args *args, uint32_t *status,
+                               verify_attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

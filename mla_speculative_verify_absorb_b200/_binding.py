@@ -63,7 +63,7 @@ _lib = None
 
 EXPORTS = (
     "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_reduce",
-    "verify_attn_build_tree_mask", "verify_attn_status", "verify_attn_strerror",
+    "verify_attn_build_tree_mask", "verify_attn_status", "verify_attn_forward_static", "verify_attn_strerror",
 )
 
 
@@ -85,6 +85,7 @@ def load_library():
             lib.verify_attn_reduce.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_build_tree_mask.argtypes = [_vp, _i32, _vp]
             lib.verify_attn_status.argtypes = [_vp, _vp, P(_u32)]
+            lib.verify_attn_forward_static.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, _vp]
             lib.verify_attn_strerror.argtypes = [ctypes.c_int]
             lib.verify_attn_strerror.restype = ctypes.c_char_p
             for name in EXPORTS[:-1]:
@@ -124,6 +125,12 @@ def verify_attn_run(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stre
 def verify_attn_reduce(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stream: int = 0):
     _check(load_library().verify_attn_reduce(ctypes.byref(plan), ctypes.byref(args), ws_ptr, ws_bytes, stream),
            "verify_attn_reduce")
+
+
+def verify_attn_forward_static(plan, args: VerifyAttnArgs, status_ptr=None, stream: int = 0):
+    """Split + reduce with the library's own fixed workspace (no allocation)."""
+    _check(load_library().verify_attn_forward_static(ctypes.byref(plan), ctypes.byref(args), status_ptr, stream),
+           "verify_attn_forward_static")
 
 
 def verify_attn_build_tree_mask(parents) -> np.ndarray:
