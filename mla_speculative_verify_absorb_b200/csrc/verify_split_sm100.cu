@@ -47,13 +47,15 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 352;          // 4 softmax + 4 KV loader + Q loader + relay + MMA warps
+constexpr int kThreads = 448;          // 4 softmax + 6 KV loader + Q loader + relay + 2 MMA warps
 constexpr int kSoftmaxThreads = 128;
 constexpr int kKvWarp0 = 4;
-constexpr int kNumKvWarps = 4;
-constexpr int kQWarp = 8;
-constexpr int kRelayWarp = 9;
-constexpr int kMmaWarp = 10;
+constexpr int kNumKvWarps = 6;
+constexpr int kQWarp = 10;
+constexpr int kRelayWarp = 11;
+constexpr int kRelayBatch = 4;          // peer stages forwarded per release-arrive instruction
+constexpr int kMmaWarp = 12;           // issues the score MMAs; also owns the TMEM allocation
+constexpr int kPvWarp = 13;            // issues the value MMAs
 
 constexpr int kStageBytes = 8192;
 constexpr int kNumStages = 14;
@@ -264,8 +266,8 @@ struct StageCursor {
   }
 };
 
-// Warps 4-7: gather the K and V stages of every tile with 16-byte cp.async.
-// Loader warp w fills global stages w, w+4, w+8, ...; each lane copies 16
+// Warps 4-9: gather the K and V stages of every tile with 16-byte cp.async.
+// Loader warp w fills global stages w, w+6, w+12, ...; each lane copies 16
 // chunks of 16 bytes (4 keys x 128 B per warp instruction) into the
 // 128-byte-swizzled stage and the hardware arrives on the CTA-local full
 // barrier once they land (leader: ring_full, peer: peer_full, relayed). The
@@ -292,20 +294,13 @@ struct KvLoader {
   }
 
   __device__ __forceinline__ void load_slots(const Segment& s, const StageDesc& d, int32_t (&sl)[16]) {
+    // All loads are issued before any value is looked at, so their latencies overlap.
     const int nkeys = d.is_v ? 8 : 16;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (j >= nkeys) break;
       const int64_t pos = key_pos(s, d, j);
-      int32_t v = -1;
-      if (pos < s.req.N) {
-        v = p.kv_indices[s.req.kv_begin + pos];
-        if (v < 0 || (int64_t)v >= p.pool_slots) {
-          atomicOr(p.status, kStatusBadSlot);
-          v = -1;
-        }
-      }
-      sl[j] = v;
+      sl[j] = pos < s.req.N ? __ldg(p.kv_indices + s.req.kv_begin + pos) : -1;
     }
   }
 
@@ -328,7 +323,8 @@ struct KvLoader {
         col = dh * 256 + (int)rank * 128 + blk * 64 + ch * 8;
         dst = base + blk * 4096 + key * 128 + ((ch ^ (key & 7)) << 4);
       }
-      const bool ok = slot_j >= 0;
+      const bool ok = slot_j >= 0 && (int64_t)slot_j < p.pool_slots;
+      if (slot_j >= 0 && !ok) atomicOr(p.status, kStatusBadSlot);
       const uint16_t* src = p.kv_pool + (ok ? (int64_t)slot_j * p.kv_stride + col : 0);
       cp_async_16(dst, src, ok ? 16u : 0u);
     }
@@ -363,9 +359,11 @@ struct KvLoader {
   }
 };
 
-// Warp 9 of the peer CTA: forwards the completion of each of its stages to the
+// Warp 11 of the peer CTA: forwards the completion of its stages to the
 // leader's ring_full after making the cp.async-written bytes visible to the
-// tensor core (async proxy).
+// tensor core (async proxy). A remote release-arrive costs hundreds of
+// cycles, so lanes 0..kRelayBatch-1 each take one stage of a batch and arrive
+// in the same instruction.
 struct Relay {
   const SplitParams& p;
   Ctrl* ctrl;
@@ -374,16 +372,21 @@ struct Relay {
   __device__ Relay(const SplitParams& p_, Ctrl* c, uint32_t r) : p(p_), ctrl(c), rank(r) {}
 
   __device__ void run(int64_t u0, int64_t u1) {
+    uint32_t total = 0;
     Segment s;
-    uint32_t st = 0;
-    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
-      const uint32_t end = st + (uint32_t)kStagesPerTile * s.n;
-      for (; st < end; ++st) {
-        const uint32_t stage = st % kNumStages;
-        if (!wait_one(smem_addr(&ctrl->peer_full[stage]), (st / kNumStages) & 1u, ctrl, p, rank)) return;
+    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) total += (uint32_t)kStagesPerTile * s.n;
+    const int lane = threadIdx.x & 31;
+    for (uint32_t st0 = 0; st0 < total; st0 += kRelayBatch) {
+      const uint32_t st = st0 + (uint32_t)lane;
+      const bool mine = lane < kRelayBatch && st < total;
+      bool ok = true;
+      if (mine) ok = wait_one(smem_addr(&ctrl->peer_full[st % kNumStages]), (st / kNumStages) & 1u, ctrl, p, rank);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      if (mine) {
         fence_proxy_async_smem();
-        mbar_arrive_cluster(map_to_rank(smem_addr(&ctrl->ring_full[stage]), 0));
+        mbar_arrive_cluster(map_to_rank(smem_addr(&ctrl->ring_full[st % kNumStages]), 0));
       }
+      __syncwarp();
     }
   }
 };
@@ -436,14 +439,27 @@ struct QLoader {
 
 // ----------------------------------------------------------------------------- MMA issuer
 
-struct Issuer {
+// Global stage index (within a segment starting at `base` with n tiles) of
+// stage k of K(i) or of V(i); the inverse of describe_stage.
+__device__ __forceinline__ uint32_t k_stage(uint32_t base, int i, int kb) {
+  return base + (i == 0 ? (uint32_t)kb : (uint32_t)(kStagesK + (i - 1) * kStagesPerTile + kb));
+}
+__device__ __forceinline__ uint32_t v_stage(uint32_t base, int n, int i, int v) {
+  return base + (i < n - 1 ? (uint32_t)(2 * kStagesK + i * kStagesPerTile + v)
+                           : (uint32_t)(kStagesK + (n - 1) * kStagesPerTile + v));
+}
+
+// Shared helpers of the two MMA-issuing threads (leader CTA only). Each
+// thread's tcgen05.commit blocks it for a few hundred cycles, so score and
+// value MMAs come from two threads in different warps: one thread's commits
+// overlap the other's MMAs.
+struct IssuerBase {
   const SplitParams& p;
   Ctrl* ctrl;
   uint8_t* smem;
   uint32_t rank, tmem;
-  uint32_t st = 0;
 
-  __device__ Issuer(const SplitParams& p_, Ctrl* c, uint8_t* s, uint32_t r, uint32_t t)
+  __device__ IssuerBase(const SplitParams& p_, Ctrl* c, uint8_t* s, uint32_t r, uint32_t t)
       : p(p_), ctrl(c), smem(s), rank(r), tmem(t) {}
 
   __device__ bool wait_bar(uint64_t* bar, uint32_t parity) {
@@ -451,64 +467,82 @@ struct Issuer {
     tc_fence_after();
     return true;
   }
+  __device__ bool wait_stage(uint32_t st) {
+    if (!wait_bar(&ctrl->ring_full[st % kNumStages], (st / kNumStages) & 1u)) return false;
+    fence_proxy_async_smem();   // cp.async-written bytes -> tensor-core reads
+    return true;
+  }
   __device__ void commit_both(uint64_t* bar) { mma_commit_2sm_mc(smem_addr(bar), (uint16_t)0x3); }
-
-  __device__ bool qk(int64_t j) {
-    const uint32_t d = tmem + kColS0 + (uint32_t)(j & 1) * 64;
-    const uint32_t q0 = smem_addr(smem + kOffQ);
-    for (int kb = 0; kb < kQBlocks; ++kb) {
-      const uint32_t stage = st % kNumStages;
-      if (!wait_bar(&ctrl->ring_full[stage], (st / kNumStages) & 1u)) return false;
-      fence_proxy_async_smem();
-      const uint32_t b0 = smem_addr(smem + kOffRing + stage * kStageBytes);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_2sm_bf16(d, sdesc_sw128(q0 + kb * 8192 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), kIdescQK,
-                     (kb | k) != 0);
-      commit_both(&ctrl->ring_empty[stage]);
-      ++st;
-    }
-    return true;
+  __device__ uint64_t stage_desc(uint32_t st, uint32_t lbo) const {
+    return sdesc_sw128(smem_addr(smem + kOffRing + (st % kNumStages) * kStageBytes), lbo, 1024);
   }
+};
 
-  __device__ bool pv(int64_t j, bool first_in_segment, int si) {
-    if (!wait_bar(&ctrl->p_full[j & 1], (uint32_t)(j >> 1) & 1u)) return false;
-    if (first_in_segment && si > 0 && !wait_bar(&ctrl->o_free, (si - 1) & 1)) return false;
-    const uint32_t pbuf = smem_addr(smem + kOffP) + (uint32_t)(j & 1) * 16384;
-    for (int kc = 0; kc < 4; ++kc) {
-      for (int dh = 0; dh < 2; ++dh) {
-        const uint32_t stage = st % kNumStages;
-        if (!wait_bar(&ctrl->ring_full[stage], (st / kNumStages) & 1u)) return false;
-        fence_proxy_async_smem();
-        const uint32_t b0 = smem_addr(smem + kOffRing + stage * kStageBytes);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const int key16 = kc * 2 + ks;   // 16-key step within the tile
-          const uint32_t a = pbuf + (key16 >> 2) * 8192 + (key16 & 3) * 32;
-          mma_2sm_bf16(tmem + kColO + dh * 128, sdesc_sw128(a, 16, 1024), sdesc_sw128(b0 + ks * 2048, 4096, 1024),
-                       kIdescPV, !(first_in_segment && kc == 0 && ks == 0));
-        }
-        commit_both(&ctrl->ring_empty[stage]);
-        ++st;
-      }
-    }
-    commit_both(&ctrl->pv_done[j & 1]);
-    return true;
-  }
+// S = Q K^T for every tile: nine K stages of four M=128, N=128, K=16 MMAs.
+struct QkIssuer : IssuerBase {
+  using IssuerBase::IssuerBase;
 
   __device__ void run(int64_t u0, int64_t u1) {
     Segment s;
     int si = 0;
     int64_t j = 0;
+    uint32_t base = 0;
+    const uint64_t qd = sdesc_sw128(smem_addr(smem + kOffQ), 16, 1024);
     for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n, ++si) {
       if (!wait_bar(&ctrl->q_full, si & 1)) return;
       for (int i = 0; i < s.n; ++i, ++j) {
-        if (!qk(j)) return;
+        // S buffer j&1 is free once the softmax of tile j-2 has signalled its P.
+        if (j >= 2 && !wait_bar(&ctrl->p_full[j & 1], (uint32_t)((j - 2) >> 1) & 1u)) return;
+        const uint32_t d = tmem + kColS0 + (uint32_t)(j & 1) * 64;
+        for (int kb = 0; kb < kQBlocks; ++kb) {
+          const uint32_t st = k_stage(base, i, kb);
+          if (!wait_stage(st)) return;
+          const uint64_t bd = stage_desc(st, 16);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_2sm_bf16(d, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
+                         (kb | k) != 0);
+          commit_both(&ctrl->ring_empty[st % kNumStages]);
+        }
         if (i == s.n - 1) commit_both(&ctrl->q_empty);
         commit_both(&ctrl->s_full[j & 1]);
-        if (i >= 1 && !pv(j - 1, i == 1, si)) return;
       }
-      if (!pv(j - 1, s.n == 1, si)) return;
+      base += (uint32_t)kStagesPerTile * s.n;
+    }
+  }
+};
+
+// O += P V for every tile: eight V stages of two M=128, N=256, K=16 MMAs.
+struct PvIssuer : IssuerBase {
+  using IssuerBase::IssuerBase;
+
+  __device__ void run(int64_t u0, int64_t u1) {
+    Segment s;
+    int si = 0;
+    int64_t j = 0;
+    uint32_t base = 0;
+    const uint64_t pd0 = sdesc_sw128(smem_addr(smem + kOffP), 16, 1024);
+    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n, ++si) {
+      for (int i = 0; i < s.n; ++i, ++j) {
+        if (!wait_bar(&ctrl->p_full[j & 1], (uint32_t)(j >> 1) & 1u)) return;
+        if (i == 0 && si > 0 && !wait_bar(&ctrl->o_free, (si - 1) & 1)) return;
+        const uint64_t pd = pd0 + (uint64_t)(((uint32_t)(j & 1) * 16384) >> 4);
+        for (int v = 0; v < kStagesV; ++v) {
+          const int kc = v >> 1, dh = v & 1;
+          const uint32_t st = v_stage(base, s.n, i, v);
+          if (!wait_stage(st)) return;
+          const uint64_t bd = stage_desc(st, 4096);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const int key16 = kc * 2 + ks;   // 16-key step within the tile
+            mma_2sm_bf16(tmem + kColO + dh * 128, pd + (uint64_t)(((key16 >> 2) * 8192 + (key16 & 3) * 32) >> 4),
+                         bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(i == 0 && kc == 0 && ks == 0));
+          }
+          commit_both(&ctrl->ring_empty[st % kNumStages]);
+        }
+        commit_both(&ctrl->pv_done[j & 1]);
+      }
+      base += (uint32_t)kStagesPerTile * s.n;
     }
   }
 };
@@ -714,7 +748,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_addr(&ctrl->q_full), 2);         // one Q loader warp per CTA
     mbar_init(smem_addr(&ctrl->q_empty), 1);
     mbar_init(smem_addr(&ctrl->o_free), 8);
-    mbar_init(smem_addr(&ctrl->mma_final), 1);
+    mbar_init(smem_addr(&ctrl->mma_final), 2);      // one commit from each issuing thread
     mbar_init(smem_addr(&ctrl->xchg), kSoftmaxThreads);
     ctrl->abort_flag = 0;
     fence_mbar_init();
@@ -741,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ld.run(u0, u1);
     cp_async_wait<0>();
   } else if (warp == kRelayWarp) {
-    if (rank == 1 && (threadIdx.x & 31) == 0) {
+    if (rank == 1) {
       Relay rl(p, ctrl, rank);
       rl.run(u0, u1);
     }
@@ -750,11 +784,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     QLoader ql(p, ctrl, smem, rank);
     ql.run(u0, u1);
     cp_async_wait<0>();
-  } else if (rank == 0) {
-    if ((threadIdx.x & 31) == 0) {
-      Issuer is(p, ctrl, smem, rank, tmem);
-      is.run(u0, u1);
-      // Everything issued so far completes before this arrives in both CTAs.
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    if (rank == 0 && (threadIdx.x & 31) == 0) {
+      if (warp == kMmaWarp) {
+        QkIssuer is(p, ctrl, smem, rank, tmem);
+        is.run(u0, u1);
+      } else {
+        PvIssuer is(p, ctrl, smem, rank, tmem);
+        is.run(u0, u1);
+      }
+      // Everything this thread issued completes before this arrives in both CTAs.
       mma_commit_2sm_mc(smem_addr(&ctrl->mma_final), (uint16_t)0x3);
     }
     __syncwarp();
