@@ -285,48 +285,60 @@ struct KvLoader {
     lane = threadIdx.x & 31;
   }
 
-  // Position (within the request) of the key this lane copies in chunk group j.
-  __device__ __forceinline__ int64_t key_pos(const Segment& s, const StageDesc& d, int j) const {
-    const int64_t kt = s.kt0 + d.tile;
-    if (!d.is_v) return kt * kKeysPerTile + rank * 64 + j * 4 + (lane >> 3);
-    const int kc = d.idx >> 1;
-    return kt * kKeysPerTile + kc * 32 + (j & 7) * 4 + (lane >> 3);
-  }
-
+  // Lane group g = lane / 8 copies a run of consecutive keys of the stage
+  // (K: 16 keys, V: 8 keys); lane & 7 selects the 16-byte chunk of the 128-byte
+  // row. One warp instruction therefore still moves four whole 128-byte rows,
+  // and each lane fetches the slots of its run with a few vector loads.
   __device__ __forceinline__ void load_slots(const Segment& s, const StageDesc& d, int32_t (&sl)[16]) {
-    // All loads are issued before any value is looked at, so their latencies overlap.
-    const int nkeys = d.is_v ? 8 : 16;
+    const int g = lane >> 3;
+    const int64_t kt = s.kt0 + d.tile;
+    const int n = d.is_v ? 8 : 16;
+    const int64_t pos0 = d.is_v ? kt * kKeysPerTile + (d.idx >> 1) * 32 + 8 * g
+                                : kt * kKeysPerTile + rank * 64 + 16 * g;
+    const int32_t* src = p.kv_indices + s.req.kv_begin + pos0;
+    if (pos0 + n <= s.req.N && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0)) {
+      const int4* v4 = reinterpret_cast<const int4*>(src);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j >= nkeys) break;
-      const int64_t pos = key_pos(s, d, j);
-      sl[j] = pos < s.req.N ? __ldg(p.kv_indices + s.req.kv_begin + pos) : -1;
+      for (int q = 0; q < 4; ++q) {
+        if (4 * q >= n) break;
+        const int4 v = __ldg(v4 + q);
+        sl[4 * q + 0] = v.x;
+        sl[4 * q + 1] = v.y;
+        sl[4 * q + 2] = v.z;
+        sl[4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j >= n) break;
+        sl[j] = pos0 + j < s.req.N ? __ldg(src + j) : -1;
+      }
     }
   }
 
   __device__ __forceinline__ void issue(const StageDesc& d, const int32_t (&sl)[16], uint32_t stage) {
     const uint32_t base = smem_addr(smem + kOffRing + stage * kStageBytes);
-    const int ch = lane & 7;
+    const int ch = lane & 7, g = lane >> 3;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       int key, col, slot_j;
       uint32_t dst;
       if (!d.is_v) {
-        key = j * 4 + (lane >> 3);
+        key = 16 * g + j;
         slot_j = sl[j];
         col = d.idx * 64 + ch * 8;
         dst = base + key * 128 + ((ch ^ (key & 7)) << 4);
       } else {
         const int blk = j >> 3, dh = d.idx & 1;
-        key = (j & 7) * 4 + (lane >> 3);
+        key = 8 * g + (j & 7);
         slot_j = sl[j & 7];
         col = dh * 256 + (int)rank * 128 + blk * 64 + ch * 8;
         dst = base + blk * 4096 + key * 128 + ((ch ^ (key & 7)) << 4);
       }
       const bool ok = slot_j >= 0 && (int64_t)slot_j < p.pool_slots;
       if (slot_j >= 0 && !ok) atomicOr(p.status, kStatusBadSlot);
-      const uint16_t* src = p.kv_pool + (ok ? (int64_t)slot_j * p.kv_stride + col : 0);
-      cp_async_16(dst, src, ok ? 16u : 0u);
+      const uint16_t* gsrc = p.kv_pool + (ok ? (int64_t)slot_j * p.kv_stride + col : 0);
+      cp_async_16(dst, gsrc, ok ? 16u : 0u);
     }
   }
 
