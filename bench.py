@@ -145,10 +145,18 @@ def cpu_baseline(inp, anc_oracle, budget_s: float = 12.0):
     order = np.random.default_rng(0).permutation(rows_total).astype(np.int64)
     chunk = max(cores, 1)
     done, t0 = 0, time.perf_counter()
-    while done < rows_total and time.perf_counter() - t0 < budget_s:
+    while done < rows_total:
         oracle.verify_rows(inp, anc_oracle, rows=order[done:done + chunk], threads=cores)
         done += chunk
-        chunk = min(chunk * 2, rows_total - done) if done < rows_total else chunk
+        spent = time.perf_counter() - t0
+        left = budget_s - spent
+        if left <= 0:
+            break
+        # next chunk: what fits in the remaining budget at the rate seen so far
+        fit = int(left / (spent / done))
+        if fit < cores:
+            break
+        chunk = min(max(cores, (fit // cores) * cores), rows_total - done)
     elapsed = time.perf_counter() - t0
     full_call_s = elapsed * rows_total / done
     value = int(inp.kv_indptr[-1]) / full_call_s
@@ -316,10 +324,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
 
-    if dist is not None:
-        t = torch.tensor([t_call, t_split, t_e2e], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_call, t_split, t_e2e = (float(x) for x in t.tolist())
+    t_call, t_split, t_e2e = max_over_ranks([t_call, t_split, t_e2e], dist, "cuda")
 
     kv = wl.total_kv
     tflops_split = flops / t_split / 1e12
@@ -364,6 +369,17 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of a list of floats over all ranks (the job's time)."""
+    import torch
+
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
 
 
 def kernel_digest() -> str:

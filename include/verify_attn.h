@@ -169,6 +169,19 @@ int verify_attn_reduce(const verify_attn_plan_t *plan, const verify_attn_args *a
 int verify_attn_build_tree_mask(const int32_t *parents_h, int32_t T, uint64_t *anc_h);
 
 /*
+ * Device version of verify_attn_build_tree_mask for a whole batch, so the
+ * mask build can run inside the same captured graph as the attention (the
+ * pages build the mask on the CPU every step: page "The Execution Phase",
+ * section "The Methodology"). parents: [sumT] request-local parent ids
+ * (root -1, otherwise 0 <= parent < node), qo_indptr: [batch+1], anc: [sumT]
+ * output. A request whose tree is malformed gets only its self bits and sets
+ * the tree bit of *status (a device status word such as the workspace's
+ * first word, or NULL). One warp per request; asynchronous, capture-safe.
+ */
+int verify_attn_build_tree_mask_device(const int32_t *parents, const int32_t *qo_indptr, int32_t batch,
+                                       uint64_t *anc, uint32_t *status, verify_attn_stream_t stream);
+
+/*
  * Read the workspace's device status word: copies it to the host on
  * `stream` and synchronises that stream (not capture-safe; call after the
  * work you want to check). Returns VERIFY_ATTN_OK, VERIFY_ATTN_DEVICE_TIMEOUT,

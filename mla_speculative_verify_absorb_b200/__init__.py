@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     lib_path,
     load_library,
     verify_attn_build_tree_mask,
+    verify_attn_build_tree_mask_device,
     verify_attn_forward_static,
     verify_attn_plan,
     verify_attn_reduce,

@@ -63,7 +63,8 @@ _lib = None
 
 EXPORTS = (
     "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_reduce",
-    "verify_attn_build_tree_mask", "verify_attn_status", "verify_attn_forward_static", "verify_attn_strerror",
+    "verify_attn_build_tree_mask", "verify_attn_build_tree_mask_device", "verify_attn_status",
+    "verify_attn_forward_static", "verify_attn_strerror",
 )
 
 
@@ -84,6 +85,7 @@ def load_library():
             lib.verify_attn_run.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_reduce.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_build_tree_mask.argtypes = [_vp, _i32, _vp]
+            lib.verify_attn_build_tree_mask_device.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp]
             lib.verify_attn_status.argtypes = [_vp, _vp, P(_u32)]
             lib.verify_attn_forward_static.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, _vp]
             lib.verify_attn_strerror.argtypes = [ctypes.c_int]
@@ -140,6 +142,13 @@ def verify_attn_build_tree_mask(parents) -> np.ndarray:
     _check(load_library().verify_attn_build_tree_mask(p.ctypes.data, int(p.shape[0]), anc.ctypes.data),
            "verify_attn_build_tree_mask")
     return anc
+
+
+def verify_attn_build_tree_mask_device(parents_ptr: int, qo_indptr_ptr: int, batch: int, anc_ptr: int,
+                                       status_ptr=None, stream: int = 0):
+    """Ancestor masks of a batch of trees on the device (asynchronous)."""
+    _check(load_library().verify_attn_build_tree_mask_device(parents_ptr, qo_indptr_ptr, int(batch), anc_ptr,
+                                                             status_ptr, stream), "verify_attn_build_tree_mask_device")
 
 
 def verify_attn_status(ws_ptr: int, stream: int = 0):

@@ -208,6 +208,16 @@ int verify_attn_build_tree_mask(const int32_t* parents_h, int32_t T, uint64_t* a
   return VERIFY_ATTN_OK;
 }
 
+int verify_attn_build_tree_mask_device(const int32_t* parents, const int32_t* qo_indptr, int32_t batch,
+                                       uint64_t* anc, uint32_t* status, verify_attn_stream_t stream) {
+  if (!parents || !qo_indptr || !anc || batch < 1) return VERIFY_ATTN_EINVAL;
+  if (va::launch_tree_mask(parents, qo_indptr, batch, anc, status, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
 int verify_attn_status(const void* ws, verify_attn_stream_t stream, uint32_t* detail_h) {
   if (!ws) return VERIFY_ATTN_EINVAL;
   uint32_t word = 0;

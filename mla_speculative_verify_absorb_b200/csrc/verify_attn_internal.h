@@ -22,6 +22,7 @@ constexpr int kRowsPerTile = 128;                // query rows per CTA pair (64 
 constexpr int kRowsPerCta = 64;
 constexpr int kKeysPerTile = 128;                // KV positions per work unit (64 per CTA for QK)
 constexpr int kWsHeaderBytes = 256;              // status word + diagnostics at ws offset 0
+constexpr int kMaxTree = VERIFY_ATTN_MAX_TREE;    // 64: one uint64 mask word per query
 
 // Status bits written (atomicOr) into the first word of the workspace.
 constexpr uint32_t kStatusTimeout = 1u << 0;      // a bounded wait expired

@@ -46,5 +46,7 @@ int split_smem_bytes();
 cudaError_t split_max_active_clusters(int* n);
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream);
 cudaError_t launch_reduce(const ReduceParams& p, cudaStream_t stream);
+cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* qo_indptr, int32_t batch, uint64_t* anc,
+                             uint32_t* status, cudaStream_t stream);
 
 }  // namespace va
