@@ -357,7 +357,7 @@ def run_gpu(args):
                      "peak_kind": f"{peak_kind} burst bf16 (cuBLAS), kernel timed alone"},
         "clocks": clock_info,
         "e2e": {"value": kv * world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,   # gather + split + reduce per call
     }
     if rank == 0 and not args.no_cpu_baseline:
         import oracle

@@ -67,7 +67,7 @@ typedef struct CUstream_st *verify_attn_stream_t;
 #define VERIFY_ATTN_D_ROPE 64
 #define VERIFY_ATTN_MAX_TREE 64
 #define VERIFY_ATTN_MAX_HEADS 1024
-#define VERIFY_ATTN_PLAN_VERSION 1
+#define VERIFY_ATTN_PLAN_VERSION 2
 
 /* Problem maxima a plan is made for (host struct, copied into the plan). */
 typedef struct {
@@ -97,14 +97,17 @@ typedef struct {
     float sm_scale;
     int32_t num_clusters;       /* persistent CTA pairs of the split kernel */
     int32_t rows_per_tile;      /* (token, head) query rows per CTA pair: 128 */
-    int32_t keys_per_tile;      /* KV positions per work unit: 128 */
+    int32_t keys_per_tile;      /* KV positions per work unit: 256 */
     int32_t row_tiles_per_req;  /* ceil(max_tree * num_heads / rows_per_tile) */
     int32_t num_slots;          /* partial-state slots in the workspace */
     int64_t ws_meta_offset;     /* bytes: float4 {m, l, count, 0} per slot row */
     int64_t ws_partial_offset;  /* bytes: fp32 O[512] per slot row */
     int64_t ws_bytes;           /* total workspace bytes */
     int32_t split_smem_bytes;   /* dynamic shared memory of the split kernel */
-    int32_t reserved[7];
+    int32_t reserved0;
+    int64_t ws_stage_offset;    /* bytes: gathered KV rows, bf16 [stage_rows, 576] */
+    int64_t stage_rows;         /* keys_per_tile * (ceil(max_total_kv / keys_per_tile) + max_batch) */
+    int32_t reserved[2];
 } verify_attn_plan_t;
 
 /* Per-call arguments (device pointers). */
@@ -142,11 +145,16 @@ int verify_attn_workspace_init(const verify_attn_plan_t *plan, void *ws, size_t 
                                verify_attn_stream_t stream);
 
 /*
- * Split kernel: every persistent CTA pair takes an equal share of the
- * (query-row tile, KV tile) units of the call, runs both contractions on the
- * tensor cores and writes one fp32 partial state (m, l, O) per (row tile,
- * pair) into ws. Asynchronous on `stream`, capture-safe. Device-side length
- * or slot errors set the status word and skip the offending work.
+ * Gather + split kernels. The gather copies the latent rows the requests
+ * reference (kv_pool rows through kv_indices) into the staging rows of ws,
+ * each request padded with zero rows to a multiple of keys_per_tile; then
+ * every persistent CTA pair takes an equal share of the (query-row tile, KV
+ * tile) units of the call, loads its tiles from the staging rows with TMA,
+ * runs both contractions on the tensor cores and writes one fp32 partial
+ * state (m, l, O) per (row tile, pair) into ws. Asynchronous on `stream`,
+ * capture-safe (two kernel launches, tensor maps encoded on the host from the
+ * ws pointer). Device-side length or slot errors set the status word and
+ * skip the offending work (a slot outside the pool reads as a zero row).
  */
 int verify_attn_run(const verify_attn_plan_t *plan, const verify_attn_args *args, void *ws,
                     size_t ws_bytes, verify_attn_stream_t stream);
@@ -194,7 +202,7 @@ int verify_attn_status(const void *ws, verify_attn_stream_t stream, uint32_t *de
 const char *verify_attn_strerror(int code);
 
 /* Size of the library-owned workspace used by verify_attn_forward_static. */
-#define VERIFY_ATTN_STATIC_WS_BYTES (32u << 20)
+#define VERIFY_ATTN_STATIC_WS_BYTES (128u << 20)
 
 /*
  * verify_attn_forward_static -- run + reduce without any allocation.
@@ -205,7 +213,7 @@ const char *verify_attn_strerror(int code);
  * heap and forbids other allocators, or a plugin that only receives the
  * tensors it may read and write. Such a caller passes its inputs and outputs
  * as for verify_attn_run / verify_attn_reduce; the scratch those kernels need
- * comes from a fixed array of VERIFY_ATTN_STATIC_WS_BYTES (32 MiB) inside the
+ * comes from a fixed array of VERIFY_ATTN_STATIC_WS_BYTES (128 MiB) inside the
  * library, which every GPU that uses the library keeps until the process
  * exits.
  *

@@ -9,6 +9,7 @@ from ._binding import (  # noqa: F401
     VERIFY_ATTN_D_LATENT,
     VERIFY_ATTN_D_ROPE,
     VERIFY_ATTN_MAX_TREE,
+    VERIFY_ATTN_STATIC_WS_BYTES,
     VerifyAttnArgs,
     VerifyAttnError,
     VerifyAttnParams,

@@ -18,6 +18,7 @@ from . import build as _build
 VERIFY_ATTN_D_LATENT = 512
 VERIFY_ATTN_D_ROPE = 64
 VERIFY_ATTN_MAX_TREE = 64
+VERIFY_ATTN_STATIC_WS_BYTES = 128 << 20
 
 _i32, _i64, _u32, _f32, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_void_p
 
@@ -36,7 +37,8 @@ class VerifyAttnPlan(ctypes.Structure):
         ("max_kv_per_req", _i64), ("max_total_kv", _i64), ("pool_slots", _i64), ("sm_scale", _f32),
         ("num_clusters", _i32), ("rows_per_tile", _i32), ("keys_per_tile", _i32), ("row_tiles_per_req", _i32),
         ("num_slots", _i32), ("ws_meta_offset", _i64), ("ws_partial_offset", _i64), ("ws_bytes", _i64),
-        ("split_smem_bytes", _i32), ("reserved", _i32 * 7),
+        ("split_smem_bytes", _i32), ("reserved0", _i32), ("ws_stage_offset", _i64), ("stage_rows", _i64),
+        ("reserved", _i32 * 2),
     ]
 
 

@@ -84,21 +84,25 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_b
 
 // ---------------------------------------------------------------- TMA
 
-// Gather four rows (row0..row3) x one box of columns starting at `col` of a
-// 2-D tensor map into consecutive box rows at `dst` (this CTA's shared
-// memory). With cta_group::2 the completed bytes are counted on the barrier
-// `cluster_bar`, which may live in the peer CTA of the pair.
-__device__ __forceinline__ void tma_gather4_2sm(uint32_t dst, const void* tmap, int32_t col, int32_t r0, int32_t r1,
-                                                int32_t r2, int32_t r3, uint32_t cluster_bar) {
+// Tiled load of one box of a 2-D tensor map at (x = column, y = row) into this
+// CTA's shared memory at `dst`. With cta_group::2 the landed bytes are counted
+// on the barrier `cluster_bar`, which may live in the peer CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_2sm(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                                uint32_t cluster_bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(cluster_bar)
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar)
       : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// Arrive on a barrier of this CTA and raise its expected transaction bytes.
+__device__ __forceinline__ void mbar_arrive_expect_tx_local(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------- cp.async

@@ -90,6 +90,10 @@ int verify_attn_plan(const verify_attn_params* params, verify_attn_plan_t* plan,
   if (clusters < 1) clusters = 1;
   const int64_t slots = clusters + (int64_t)q.max_batch * row_tiles;
   if (slots > INT32_MAX) return VERIFY_ATTN_UNSUPPORTED;
+  // Staging rows: every request padded to whole key tiles (TMA row
+  // coordinates are 32-bit).
+  const int64_t stage_rows = key_tiles_total * va::kKeysPerTile;
+  if (stage_rows > INT32_MAX) return VERIFY_ATTN_UNSUPPORTED;
 
   memset(plan, 0, sizeof(*plan));
   plan->version = VERIFY_ATTN_PLAN_VERSION;
@@ -107,7 +111,9 @@ int verify_attn_plan(const verify_attn_params* params, verify_attn_plan_t* plan,
   plan->num_slots = (int32_t)slots;
   plan->ws_meta_offset = va::kWsHeaderBytes;
   plan->ws_partial_offset = round_up(plan->ws_meta_offset + slots * va::kRowsPerTile * 16, kAlign);
-  plan->ws_bytes = plan->ws_partial_offset + slots * va::kRowsPerTile * va::kDLatent * 4;
+  plan->ws_stage_offset = round_up(plan->ws_partial_offset + slots * va::kRowsPerTile * va::kDLatent * 4, 1024);
+  plan->stage_rows = stage_rows;
+  plan->ws_bytes = plan->ws_stage_offset + stage_rows * va::kDQK * 2;
   plan->split_smem_bytes = va::split_smem_bytes();
   *ws_bytes = (size_t)plan->ws_bytes;
   return VERIFY_ATTN_OK;
@@ -155,7 +161,27 @@ int verify_attn_run(const verify_attn_plan_t* plan, const verify_attn_args* a, v
   p.status = reinterpret_cast<uint32_t*>(base);
   p.meta = reinterpret_cast<float4*>(base + plan->ws_meta_offset);
   p.partial = reinterpret_cast<float*>(base + plan->ws_partial_offset);
-  if (va::launch_split(p, (cudaStream_t)stream) != cudaSuccess) {
+  p.stage = reinterpret_cast<const uint16_t*>(base + plan->ws_stage_offset);
+  p.stage_rows = plan->stage_rows;
+
+  va::GatherParams gp;
+  gp.kv_pool = a->kv_pool;
+  gp.kv_stride = a->kv_row_stride;
+  gp.kv_indices = a->kv_indices;
+  gp.kv_indptr = a->kv_indptr;
+  gp.qo_indptr = a->qo_indptr;
+  gp.batch = a->batch;
+  gp.max_tree = plan->max_tree;
+  gp.max_kv_per_req = plan->max_kv_per_req;
+  gp.pool_slots = plan->pool_slots;
+  gp.status = p.status;
+  gp.stage = reinterpret_cast<uint16_t*>(base + plan->ws_stage_offset);
+  // A grid of a few CTAs per SM loops over the key tiles of the call.
+  const int64_t tiles = plan->stage_rows / va::kKeysPerTile;
+  gp.stage_tiles = tiles;
+  const int64_t grid = tiles < (int64_t)plan->num_clusters * 8 ? tiles : (int64_t)plan->num_clusters * 8;
+  if (va::launch_gather(gp, (int)grid, (cudaStream_t)stream) != cudaSuccess ||
+      va::launch_split(p, (cudaStream_t)stream) != cudaSuccess) {
     cudaGetLastError();
     return VERIFY_ATTN_CUDA_ERROR;
   }

@@ -20,7 +20,7 @@ constexpr int kDRope = VERIFY_ATTN_D_ROPE;       // 64: rope width
 constexpr int kDQK = kDLatent + kDRope;          // 576: score contraction width
 constexpr int kRowsPerTile = 128;                // query rows per CTA pair (64 per CTA)
 constexpr int kRowsPerCta = 64;
-constexpr int kKeysPerTile = 128;                // KV positions per work unit (64 per CTA for QK)
+constexpr int kKeysPerTile = 256;                // KV positions per work unit (128 per CTA for QK)
 constexpr int kWsHeaderBytes = 256;              // status word + diagnostics at ws offset 0
 constexpr int kMaxTree = VERIFY_ATTN_MAX_TREE;    // 64: one uint64 mask word per query
 

@@ -24,6 +24,22 @@ struct SplitParams {
   uint32_t* status;          // workspace status word
   float4* meta;              // [num_slots, 128] {m, l, count, 0}
   float* partial;            // [num_slots, 128, 512]
+  const uint16_t* stage;     // [stage_rows, 576] gathered KV rows (verify_gather.cu)
+  int64_t stage_rows;
+};
+
+// KV gather into the staging rows of the workspace.
+struct GatherParams {
+  const uint16_t* kv_pool;
+  int64_t kv_stride;
+  const int32_t* kv_indices;
+  const int32_t* kv_indptr;
+  const int32_t* qo_indptr;
+  int32_t batch, max_tree;
+  int64_t max_kv_per_req, pool_slots;
+  uint32_t* status;
+  uint16_t* stage;
+  int64_t stage_tiles;       // capacity of `stage` in key tiles
 };
 
 struct ReduceParams {
@@ -45,6 +61,7 @@ struct ReduceParams {
 int split_smem_bytes();
 cudaError_t split_max_active_clusters(int* n);
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream);
+cudaError_t launch_gather(const GatherParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_reduce(const ReduceParams& p, cudaStream_t stream);
 cudaError_t launch_tree_mask(const int32_t* parents, const int32_t* qo_indptr, int32_t batch, uint64_t* anc,
                              uint32_t* status, cudaStream_t stream);

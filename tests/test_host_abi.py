@@ -46,20 +46,24 @@ def _params(**kw):
 
 def test_plan_long_context_layout():
     plan, ws = va.verify_attn_plan(_params())
-    assert plan.version == 1
+    assert plan.version == 2
     assert plan.num_clusters == 74                  # one CTA pair per two SMs
     assert plan.row_tiles_per_req == 32             # 64 nodes x 64 heads / 128
     assert plan.num_slots == 74 + 32
     assert plan.ws_meta_offset == 256
     assert plan.ws_partial_offset % 256 == 0
-    assert ws == plan.ws_bytes == plan.ws_partial_offset + plan.num_slots * 128 * 512 * 4
+    assert plan.keys_per_tile == 256
+    assert plan.ws_stage_offset % 1024 == 0
+    assert plan.ws_stage_offset >= plan.ws_partial_offset + plan.num_slots * 128 * 512 * 4
+    assert plan.stage_rows == 256 * ((65600 + 255) // 256 + 1)   # whole key tiles, one spare per request
+    assert ws == plan.ws_bytes == plan.ws_stage_offset + plan.stage_rows * 576 * 2
     assert 0 < plan.split_smem_bytes <= 232448
 
 
 def test_plan_caps_clusters_by_work():
     plan, _ = va.verify_attn_plan(_params(num_heads=8, max_tree=4, max_kv_per_req=260, max_total_kv=260,
                                           pool_slots=4096))
-    assert plan.num_clusters == 3                   # 1 row tile x 3 key tiles
+    assert plan.num_clusters == 2                   # 1 row tile x 2 key tiles of 256
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -13,7 +13,7 @@ import pytest
 import mla_speculative_verify_absorb_b200 as va
 from workloads import WORKLOADS
 
-ROWS, KEYS = 128, 128
+ROWS, KEYS = 128, 256
 
 
 def _requests(T_list, N_list, H):

@@ -36,7 +36,7 @@ def test_static_workspace_matches_allocated_workspace(name):
     inp = generate(wl)
     anc = product_anc(inp)
     attn = make_attention(wl)
-    assert attn.ws_bytes <= (32 << 20)
+    assert attn.ws_bytes <= va.VERIFY_ATTN_STATIC_WS_BYTES
 
     ref = wdev.to_device(inp, anc)
     attn(*wdev.positional(ref), lse=ref["lse"], visible_count=ref["visible_count"])
@@ -65,7 +65,7 @@ def test_static_workspace_rejects_large_plans():
                                  d_latent=512, d_rope=64, num_sms=0, max_kv_per_req=max(wl.kv_lens),
                                  max_total_kv=wl.total_kv, pool_slots=wl.pool_slots, sm_scale=wl.sm_scale)
     plan, ws = va.verify_attn_plan(params)
-    assert ws > (32 << 20)
+    assert ws > va.VERIFY_ATTN_STATIC_WS_BYTES
     args = va.VerifyAttnArgs()
     with pytest.raises(va.VerifyAttnError) as e:
         va.verify_attn_forward_static(plan, args, None, 0)
