@@ -228,37 +228,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ----------------------------------------------------------------------------- producers
 
 // Stage order of one segment of n tiles, shared by the producers and the MMA
-// issuers: K(0), then for i = 1..n-1: K(i), V(i-1), then V(n-1). K(i) is 9
+// issuer: K(0), then for i = 1..n-1: K(i), V(i-1), then V(n-1). K(i) is 9
 // stages (one 64-column block of the 576 score columns for the CTA's 128
 // keys), V(i) 8 stages (64 keys x two 64-column blocks of the CTA's value
 // columns; stage v covers keys 64 (v >> 1) .. +63 and blocks 2 (v & 1), +1),
 // so a segment has 17 n stages.
 constexpr int kStagesK = kQBlocks;    // 9
 constexpr int kStagesV = 8;
-constexpr int kStagesPerTile = kStagesK + kStagesV;
-
-struct StageDesc {
-  int32_t tile;    // tile index within the segment
-  int32_t is_v;    // 0: K stage, 1: V stage
-  int32_t idx;     // K: column block 0..8; V: 2 * key quarter + value half
-};
-
-__device__ __forceinline__ StageDesc describe_stage(uint32_t p, int n) {
-  StageDesc d;
-  if (p < (uint32_t)kStagesK) {
-    d.tile = 0; d.is_v = 0; d.idx = (int)p;
-    return d;
-  }
-  const uint32_t q = p - kStagesK;
-  const uint32_t blk = q / kStagesPerTile, r = q % kStagesPerTile;
-  if (blk < (uint32_t)(n - 1)) {
-    if (r < (uint32_t)kStagesK) { d.tile = (int)blk + 1; d.is_v = 0; d.idx = (int)r; }
-    else { d.tile = (int)blk; d.is_v = 1; d.idx = (int)r - kStagesK; }
-  } else {
-    d.tile = n - 1; d.is_v = 1; d.idx = (int)(q - (uint32_t)(n - 1) * kStagesPerTile);
-  }
-  return d;
-}
 
 // Warp 4, one thread per CTA: walks the cluster's stages in order and loads
 // each into the ring with tiled TMA copies from the staging rows. K stage of
@@ -273,30 +249,50 @@ struct Producer {
   uint32_t rank;
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
+  uint32_t st = 0;
+
+  // Next ring slot: wait until the MMAs of its previous use completed, then
+  // (leader) announce the bytes both CTAs will land on its full barrier.
+  __device__ bool acquire(uint32_t& dst, uint32_t& bar) {
+    const uint32_t stage = st % kNumStages, use = st / kNumStages;
+    if (use >= 1 && !wait_one(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return false;
+    const uint32_t full = smem_addr(&ctrl->ring_full[stage]);
+    if (rank == 0) mbar_arrive_expect_tx_local(full, 2u * kStageBytes);
+    bar = map_to_rank(full, 0);
+    dst = smem_addr(smem + kOffRing + stage * kStageBytes);
+    ++st;
+    return true;
+  }
+  __device__ bool load_k(int32_t row0) {
+    for (int kb = 0; kb < kStagesK; ++kb) {
+      uint32_t dst, bar;
+      if (!acquire(dst, bar)) return false;
+      tma_load_2d_2sm(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar);
+    }
+    return true;
+  }
+  __device__ bool load_v(int32_t row0) {
+    for (int v = 0; v < kStagesV; ++v) {
+      uint32_t dst, bar;
+      if (!acquire(dst, bar)) return false;
+      const int32_t key = row0 + 64 * (v >> 1);
+      const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
+      tma_load_2d_2sm(dst, tm_v, col, key, bar);
+      tma_load_2d_2sm(dst + 8192, tm_v, col + 64, key, bar);
+    }
+    return true;
+  }
 
   __device__ void run(int64_t u0, int64_t u1) {
     Segment s;
-    uint32_t st = 0;
     for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
-      const int nst = kStagesPerTile * s.n;
-      for (int q = 0; q < nst; ++q, ++st) {
-        const StageDesc d = describe_stage((uint32_t)q, s.n);
-        const uint32_t stage = st % kNumStages, use = st / kNumStages;
-        if (use >= 1 && !wait_one(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return;
-        const uint32_t full = smem_addr(&ctrl->ring_full[stage]);
-        if (rank == 0) mbar_arrive_expect_tx_local(full, 2u * kStageBytes);
-        const uint32_t bar = map_to_rank(full, 0);
-        const uint32_t dst = smem_addr(smem + kOffRing + stage * kStageBytes);
-        const int32_t row0 = (s.kt_base + s.kt0 + d.tile) * kKeysPerTile;
-        if (!d.is_v) {
-          tma_load_2d_2sm(dst, tm_k, 64 * d.idx, row0 + 128 * (int32_t)rank, bar);
-        } else {
-          const int32_t key = row0 + 64 * (d.idx >> 1);
-          const int32_t col = 256 * (int32_t)rank + 128 * (d.idx & 1);
-          tma_load_2d_2sm(dst, tm_v, col, key, bar);
-          tma_load_2d_2sm(dst + 8192, tm_v, col + 64, key, bar);
-        }
+      const int32_t row0 = (s.kt_base + s.kt0) * kKeysPerTile;
+      if (!load_k(row0)) return;
+      for (int i = 1; i < s.n; ++i) {
+        if (!load_k(row0 + i * kKeysPerTile)) return;
+        if (!load_v(row0 + (i - 1) * kKeysPerTile)) return;
       }
+      if (!load_v(row0 + (s.n - 1) * kKeysPerTile)) return;
     }
   }
 };
@@ -363,63 +359,83 @@ struct Issuer {
   Ctrl* ctrl;
   uint8_t* smem;
   uint32_t rank, tmem;
+  uint32_t st = 0;
+  uint64_t qd = 0, pd = 0;
 
   __device__ bool wait_bar(uint64_t* bar, uint32_t parity) {
     if (!wait_one(smem_addr(bar), parity, ctrl, p, rank)) return false;
     tc_fence_after();
     return true;
   }
+  // A ring stage is usually landed or about to: poll it without sleeping
+  // before falling back to the bounded wait.
+  __device__ bool wait_stage(uint32_t& saddr) {
+    const uint32_t stage = st % kNumStages, parity = (st / kNumStages) & 1u;
+    const uint32_t bar = smem_addr(&ctrl->ring_full[stage]);
+    bool ok = false;
+    for (int spin = 0; spin < 256 && !ok; ++spin) ok = mbar_test_wait_cta(bar, parity);
+    if (!ok && !wait_one(bar, parity, ctrl, p, rank)) return false;
+    saddr = smem_addr(smem + kOffRing + stage * kStageBytes);
+    return true;
+  }
+  __device__ void release_stage() {
+    mma_commit_2sm_mc(smem_addr(&ctrl->ring_empty[st % kNumStages]), (uint16_t)0x3);
+    ++st;
+  }
   __device__ void commit_both(uint64_t* bar) { mma_commit_2sm_mc(smem_addr(bar), (uint16_t)0x3); }
+
+  // S(j) = Q K(j)^T from the nine K stages of tile j.
+  __device__ bool score(int64_t j, bool last_of_segment) {
+    // S buffer j&1 is free once the softmax warps have read S of tile j-2.
+    if (j >= 2 && !wait_bar(&ctrl->s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u)) return false;
+    const uint32_t dt = tmem + kColS0 + (uint32_t)(j & 1) * 128;
+    for (int kb = 0; kb < kStagesK; ++kb) {
+      uint32_t saddr;
+      if (!wait_stage(saddr)) return false;
+      const uint64_t bd = sdesc_sw128(saddr, 16, 1024);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_2sm_bf16(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
+                     (kb | k) != 0);
+      release_stage();
+    }
+    if (last_of_segment) commit_both(&ctrl->q_empty);
+    commit_both(&ctrl->s_full[j & 1]);
+    return true;
+  }
+  // O += P(j) V(j) from the eight V stages of tile j.
+  __device__ bool value(int64_t j, bool first_of_segment, int si) {
+    if (!wait_bar(&ctrl->p_full, (uint32_t)(j & 1))) return false;
+    if (first_of_segment && si > 0 && !wait_bar(&ctrl->o_free, (si - 1) & 1)) return false;
+    for (int v = 0; v < kStagesV; ++v) {
+      uint32_t saddr;
+      if (!wait_stage(saddr)) return false;
+      const int kq = v >> 1, dh = v & 1;
+      const uint64_t bd = sdesc_sw128(saddr, 8192, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_2sm_bf16(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
+                     bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(first_of_segment && kq == 0 && ks == 0));
+      release_stage();
+    }
+    commit_both(&ctrl->pv_done);
+    return true;
+  }
 
   __device__ void run(int64_t u0, int64_t u1) {
     Segment s;
     int si = 0;
-    int64_t jbase = 0;   // global index of the segment's first tile
-    uint32_t st = 0;
-    const uint64_t qd = sdesc_sw128(smem_addr(smem + kOffQ), 16, 1024);
-    const uint64_t pd = sdesc_sw128(smem_addr(smem + kOffP), 16, 1024);
-    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n, ++si) {
-      const int nst = kStagesPerTile * s.n;
-      for (int q = 0; q < nst; ++q, ++st) {
-        const StageDesc d = describe_stage((uint32_t)q, s.n);
-        const int64_t j = jbase + d.tile;
-        const uint32_t saddr = smem_addr(smem + kOffRing + (st % kNumStages) * kStageBytes);
-        if (!d.is_v) {
-          if (d.idx == 0) {
-            if (d.tile == 0 && !wait_bar(&ctrl->q_full, si & 1)) return;
-            // S buffer j&1 is free once the softmax warps have read S of tile j-2.
-            if (j >= 2 && !wait_bar(&ctrl->s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u)) return;
-          }
-          if (!wait_bar(&ctrl->ring_full[st % kNumStages], (st / kNumStages) & 1u)) return;
-          const uint32_t dt = tmem + kColS0 + (uint32_t)(j & 1) * 128;
-          const uint64_t bd = sdesc_sw128(saddr, 16, 1024);
-          const int kb = d.idx;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_2sm_bf16(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
-                         (kb | k) != 0);
-          commit_both(&ctrl->ring_empty[st % kNumStages]);
-          if (kb == kStagesK - 1) {
-            if (d.tile == s.n - 1) commit_both(&ctrl->q_empty);
-            commit_both(&ctrl->s_full[j & 1]);
-          }
-        } else {
-          if (d.idx == 0) {
-            if (!wait_bar(&ctrl->p_full, (uint32_t)(j & 1))) return;
-            if (d.tile == 0 && si > 0 && !wait_bar(&ctrl->o_free, (si - 1) & 1)) return;
-          }
-          if (!wait_bar(&ctrl->ring_full[st % kNumStages], (st / kNumStages) & 1u)) return;
-          const int kq = d.idx >> 1, dh = d.idx & 1;
-          const uint64_t bd = sdesc_sw128(saddr, 8192, 1024);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_2sm_bf16(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
-                         bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(d.tile == 0 && kq == 0 && ks == 0));
-          commit_both(&ctrl->ring_empty[st % kNumStages]);
-          if (d.idx == kStagesV - 1) commit_both(&ctrl->pv_done);
-        }
+    int64_t j = 0;   // global index of the segment's first tile
+    qd = sdesc_sw128(smem_addr(smem + kOffQ), 16, 1024);
+    pd = sdesc_sw128(smem_addr(smem + kOffP), 16, 1024);
+    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n, ++si, j += s.n) {
+      if (!wait_bar(&ctrl->q_full, si & 1)) return;
+      if (!score(j, s.n == 1)) return;
+      for (int i = 1; i < s.n; ++i) {
+        if (!score(j + i, i == s.n - 1)) return;
+        if (!value(j + i - 1, i == 1, si)) return;
       }
-      jbase += s.n;
+      if (!value(j + s.n - 1, s.n == 1, si)) return;
     }
   }
 };
