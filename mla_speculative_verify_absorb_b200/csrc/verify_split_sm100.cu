@@ -28,9 +28,11 @@
 //    per instruction, K = keys; CTA r supplies value columns [256 r, 256 r +
 //    256), so each CTA loads half of every V row. Both contractions run at
 //    N = 256, the shape at which the pair's tensor cores stay saturated.
-//  * One thread per CTA issues the TMA copies into a ring of 16 KB stages,
+//  * One warp per CTA issues the TMA copies into a ring of 16 KB stages,
 //    counting both CTAs' bytes on the leader's barrier (cta_group::2); one
-//    thread of the leader issues every MMA of the pair; four softmax
+//    warp of the leader issues every MMA of the pair (both run converged,
+//    with one elected lane executing each copy, MMA and commit, so their
+//    operands stay warp-uniform); four softmax
 //    warps per CTA read S from TMEM, apply scale and the ancestor mask, keep
 //    the online softmax (the O rescale is skipped unless the row max grows
 //    by more than 2^8), write bf16 P into shared memory and finally dump O
@@ -56,7 +58,7 @@ using namespace ptx;
 
 constexpr int kThreads = 224;          // 4 softmax + TMA producer + Q loader + MMA warps
 constexpr int kSoftmaxThreads = 128;
-constexpr int kProdWarp = 4;           // one thread issues the K/V TMA copies of its CTA
+constexpr int kProdWarp = 4;           // issues the K/V TMA copies of its CTA
 constexpr int kQWarp = 5;
 constexpr int kMmaWarp = 6;            // issues all MMAs; also owns the TMEM allocation
 
@@ -236,7 +238,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 constexpr int kStagesK = kQBlocks;    // 9
 constexpr int kStagesV = 8;
 
-// Warp 4, one thread per CTA: walks the cluster's stages in order and loads
+// Warp 4 of each CTA: walks the cluster's stages in order and loads
 // each into the ring with tiled TMA copies from the staging rows. K stage of
 // block kb: box [128 keys x 64 columns] at column 64 kb, keys 128 r .. of the
 // tile (CTA r). V stage: two boxes [64 keys x 64 columns] at value columns
@@ -253,11 +255,17 @@ struct Producer {
 
   // Next ring slot: wait until the MMAs of its previous use completed, then
   // (leader) announce the bytes both CTAs will land on its full barrier.
+  // The whole warp runs this; one elected lane issues each instruction.
   __device__ bool acquire(uint32_t& dst, uint32_t& bar) {
     const uint32_t stage = st % kNumStages, use = st / kNumStages;
-    if (use >= 1 && !wait_one(smem_addr(&ctrl->ring_empty[stage]), (use - 1) & 1u, ctrl, p, rank)) return false;
+    if (use >= 1) {
+      const uint32_t e = smem_addr(&ctrl->ring_empty[stage]), par = (use - 1) & 1u;
+      bool ok = false;
+      for (int spin = 0; spin < 64 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(e, par));
+      if (!ok && !wait_warp(e, par, ctrl, p, rank)) return false;
+    }
     const uint32_t full = smem_addr(&ctrl->ring_full[stage]);
-    if (rank == 0) mbar_arrive_expect_tx_local(full, 2u * kStageBytes);
+    if (rank == 0) mbar_arrive_expect_tx_local_elect(full, 2u * kStageBytes);
     bar = map_to_rank(full, 0);
     dst = smem_addr(smem + kOffRing + stage * kStageBytes);
     ++st;
@@ -267,7 +275,7 @@ struct Producer {
     for (int kb = 0; kb < kStagesK; ++kb) {
       uint32_t dst, bar;
       if (!acquire(dst, bar)) return false;
-      tma_load_2d_2sm(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar);
+      tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar);
     }
     return true;
   }
@@ -277,8 +285,8 @@ struct Producer {
       if (!acquire(dst, bar)) return false;
       const int32_t key = row0 + 64 * (v >> 1);
       const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
-      tma_load_2d_2sm(dst, tm_v, col, key, bar);
-      tma_load_2d_2sm(dst + 8192, tm_v, col + 64, key, bar);
+      tma_load_2d_2sm_elect(dst, tm_v, col, key, bar);
+      tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar);
     }
     return true;
   }
@@ -345,9 +353,10 @@ struct QLoader {
 
 // ----------------------------------------------------------------------------- MMA issuers
 
-// The MMA issuer: one thread of the leader CTA issues every tcgen05.mma of
-// the pair, in ring order, so the two SMs' tensor cores always see one
-// instruction stream. For each stage: K stage of tile i -> four M=128, N=256,
+// The MMA issuer: warp 6 of the leader CTA issues every tcgen05.mma of the
+// pair, in ring order, so the two SMs' tensor cores always see one
+// instruction stream (two issuing threads interleaving pair MMAs were seen
+// to hang the pair). For each stage: K stage of tile i -> four M=128, N=256,
 // K=16 score MMAs into S buffer (j & 1); V stage -> four value MMAs into one
 // half of O. Before the first K stage of a tile it waits until the softmax
 // warps have read S of tile j-2 from that buffer (and at a segment start for
@@ -363,7 +372,7 @@ struct Issuer {
   uint64_t qd = 0, pd = 0;
 
   __device__ bool wait_bar(uint64_t* bar, uint32_t parity) {
-    if (!wait_one(smem_addr(bar), parity, ctrl, p, rank)) return false;
+    if (!wait_warp(smem_addr(bar), parity, ctrl, p, rank)) return false;
     tc_fence_after();
     return true;
   }
@@ -373,16 +382,16 @@ struct Issuer {
     const uint32_t stage = st % kNumStages, parity = (st / kNumStages) & 1u;
     const uint32_t bar = smem_addr(&ctrl->ring_full[stage]);
     bool ok = false;
-    for (int spin = 0; spin < 256 && !ok; ++spin) ok = mbar_test_wait_cta(bar, parity);
-    if (!ok && !wait_one(bar, parity, ctrl, p, rank)) return false;
+    for (int spin = 0; spin < 256 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(bar, parity));
+    if (!ok && !wait_warp(bar, parity, ctrl, p, rank)) return false;
     saddr = smem_addr(smem + kOffRing + stage * kStageBytes);
     return true;
   }
   __device__ void release_stage() {
-    mma_commit_2sm_mc(smem_addr(&ctrl->ring_empty[st % kNumStages]), (uint16_t)0x3);
+    mma_commit_2sm_mc_elect(smem_addr(&ctrl->ring_empty[st % kNumStages]), (uint16_t)0x3);
     ++st;
   }
-  __device__ void commit_both(uint64_t* bar) { mma_commit_2sm_mc(smem_addr(bar), (uint16_t)0x3); }
+  __device__ void commit_both(uint64_t* bar) { mma_commit_2sm_mc_elect(smem_addr(bar), (uint16_t)0x3); }
 
   // S(j) = Q K(j)^T from the nine K stages of tile j.
   __device__ bool score(int64_t j, bool last_of_segment) {
@@ -395,8 +404,8 @@ struct Issuer {
       const uint64_t bd = sdesc_sw128(saddr, 16, 1024);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_2sm_bf16(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
-                     (kb | k) != 0);
+        mma_2sm_bf16_elect(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
+                           (kb | k) != 0);
       release_stage();
     }
     if (last_of_segment) commit_both(&ctrl->q_empty);
@@ -414,8 +423,8 @@ struct Issuer {
       const uint64_t bd = sdesc_sw128(saddr, 8192, 1024);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        mma_2sm_bf16(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
-                     bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(first_of_segment && kq == 0 && ks == 0));
+        mma_2sm_bf16_elect(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
+                           bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(first_of_segment && kq == 0 && ks == 0));
       release_stage();
     }
     commit_both(&ctrl->pv_done);
@@ -669,15 +678,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
   } else if (warp == kProdWarp) {
-    if ((threadIdx.x & 31) == 0) {
-      Producer pr{p, ctrl, smem, rank, &tm_k, &tm_v};
-      pr.run(u0, u1);
-      // After an abort, copies issued before it may still be in flight:
-      // give them time to land before the CTA can exit.
-      if (*(volatile int32_t*)&ctrl->abort_flag) {
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < kDrainNs) {
-        }
+    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_v};
+    pr.run(u0, u1);
+    // After an abort, copies issued before it may still be in flight:
+    // give them time to land before the CTA can exit.
+    if ((threadIdx.x & 31) == 0 && *(volatile int32_t*)&ctrl->abort_flag) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < kDrainNs) {
       }
     }
     __syncwarp();
@@ -686,11 +693,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ql.run(u0, u1);
     cp_async_wait<0>();
   } else if (warp == kMmaWarp) {
-    if (rank == 0 && (threadIdx.x & 31) == 0) {
+    if (rank == 0) {
       Issuer is{p, ctrl, smem, rank, tmem};
       is.run(u0, u1);
-      // Everything this thread issued completes before this arrives in both CTAs.
-      mma_commit_2sm_mc(smem_addr(&ctrl->mma_final), (uint16_t)0x3);
+      // Everything the warp issued completes before this arrives in both CTAs.
+      mma_commit_2sm_mc_elect(smem_addr(&ctrl->mma_final), (uint16_t)0x3);
     }
     __syncwarp();
   }
