@@ -111,15 +111,24 @@ __device__ __forceinline__ void tma_load_2d_2sm(uint32_t dst, const void* tmap, 
       : "memory");
 }
 
-// tma_load_2d_2sm by one elected lane of a converged warp.
+// L2 policy that keeps lines in L2 ahead of normally cached data (for tiles
+// that many CTAs re-read).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_2d_2sm by one elected lane of a converged warp, with an L2 cache
+// policy for the loaded lines.
 __device__ __forceinline__ void tma_load_2d_2sm_elect(uint32_t dst, const void* tmap, int32_t x, int32_t y,
-                                                      uint32_t cluster_bar) {
+                                                      uint32_t cluster_bar, uint64_t policy) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
       "elect.sync r|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];\n\t}" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar)
+      "@e cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar), "l"(policy)
       : "memory");
 }
 

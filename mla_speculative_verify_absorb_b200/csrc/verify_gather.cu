@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kGatherThreads) verify_gather_kernel(const Gat
         for (int c = 0; c < 3; ++c) {
           const int e = lane + 32 * c;
           v[q][c] = make_int4(0, 0, 0, 0);
-          if (s >= 0 && e < kRowVecs) v[q][c] = __ldg(src + e);
+          if (s >= 0 && e < kRowVecs) v[q][c] = __ldcs(src + e);   // read once: stream past L2
         }
       }
 #pragma unroll

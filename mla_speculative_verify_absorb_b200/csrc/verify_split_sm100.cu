@@ -252,6 +252,7 @@ struct Producer {
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
   uint32_t st = 0;
+  uint64_t policy = l2_policy_evict_last();   // every K/V tile is re-read by all row tiles
 
   // Next ring slot: wait until the MMAs of its previous use completed, then
   // (leader) announce the bytes both CTAs will land on its full barrier.
@@ -275,7 +276,7 @@ struct Producer {
     for (int kb = 0; kb < kStagesK; ++kb) {
       uint32_t dst, bar;
       if (!acquire(dst, bar)) return false;
-      tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar);
+      tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar, policy);
     }
     return true;
   }
@@ -285,8 +286,8 @@ struct Producer {
       if (!acquire(dst, bar)) return false;
       const int32_t key = row0 + 64 * (v >> 1);
       const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
-      tma_load_2d_2sm_elect(dst, tm_v, col, key, bar);
-      tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar);
+      tma_load_2d_2sm_elect(dst, tm_v, col, key, bar, policy);
+      tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar, policy);
     }
     return true;
   }
@@ -541,17 +542,29 @@ struct Softmax {
 
         const uint64_t vis0 = valid_row ? visible_bits(key0, L, N, anc) : 0ull;
         const uint64_t vis1 = valid_row ? visible_bits(key0 + 64, L, N, anc) : 0ull;
-        float mx = -CUDART_INF_F;
+        // Row max of the raw scores (the scale is positive, so it commutes
+        // with max), over eight independent chains; masked keys become -inf.
+        // Tiles inside the prefix are fully visible for the whole warp.
+        float mk[8];
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const uint64_t vis = e < 64 ? vis0 : vis1;
-          const float x = ((vis >> (e & 63)) & 1ull) ? __uint_as_float(v[e]) * scale : -CUDART_INF_F;
-          v[e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+        for (int k = 0; k < 8; ++k) mk[k] = -CUDART_INF_F;
+        if (__all_sync(0xffffffffu, (vis0 & vis1) == ~0ull)) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            const uint64_t vis = e < 64 ? vis0 : vis1;
+            const float x = ((vis >> (e & 63)) & 1ull) ? __uint_as_float(v[e]) : -CUDART_INF_F;
+            v[e] = __float_as_uint(x);
+            mk[e & 7] = fmaxf(mk[e & 7], x);
+          }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                               fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
         float mx_other;
         if (!exchange(mx, mx_other)) return false;
-        const float m_tile = fmaxf(mx, mx_other);
+        const float m_tile = fmaxf(mx, mx_other) * scale;
 
         float alpha = 1.f;
         bool rescale = false;
@@ -564,15 +577,22 @@ struct Softmax {
         }
         const float m_use = (m_run == -CUDART_INF_F) ? 0.f : m_run;
 
-        float lsum = 0.f;
+        // p = 2^(s * scale - m): one packed FMA per two keys, then the
+        // exponentials; the row sum over four packed chains.
+        const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m_use, -m_use);
+        float2 sum2[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sum2[k] = make_float2(0.f, 0.f);
         uint32_t w[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
-          const float p0 = exp2f(__uint_as_float(v[2 * e]) - m_use);
-          const float p1 = exp2f(__uint_as_float(v[2 * e + 1]) - m_use);
-          lsum += p0 + p1;
-          w[e] = pack_bf16x2(p0, p1);
+          const float2 a = __ffma2_rn(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, nm2);
+          const float2 pe = make_float2(exp2f(a.x), exp2f(a.y));
+          sum2[e & 3] = __fadd2_rn(sum2[e & 3], pe);
+          w[e] = pack_bf16x2(pe.x, pe.y);
         }
+        const float2 s01 = __fadd2_rn(sum2[0], sum2[1]), s23 = __fadd2_rn(sum2[2], sum2[3]);
+        const float lsum = (s01.x + s01.y) + (s23.x + s23.y);
         l_run = l_run * alpha + lsum;
         cnt += (float)(__popcll(vis0) + __popcll(vis1));
 
