@@ -142,6 +142,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_local_elect(uint32_t bar, 
       : "memory");
 }
 
+// tma_load_2d_2sm with an L2 cache policy for the loaded lines.
+__device__ __forceinline__ void tma_load_2d_2sm(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                                uint32_t cluster_bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

@@ -28,11 +28,13 @@
 //    per instruction, K = keys; CTA r supplies value columns [256 r, 256 r +
 //    256), so each CTA loads half of every V row. Both contractions run at
 //    N = 256, the shape at which the pair's tensor cores stay saturated.
-//  * One warp per CTA issues the TMA copies into a ring of 16 KB stages,
-//    counting both CTAs' bytes on the leader's barrier (cta_group::2); one
-//    warp of the leader issues every MMA of the pair (both run converged,
-//    with one elected lane executing each copy, MMA and commit, so their
-//    operands stay warp-uniform); four softmax
+//  * Two warps per CTA issue the TMA copies into a ring of 16 KB stages,
+//    taking alternate stages (bulk copies issued by one thread complete one
+//    after another, so a single issuing thread cannot keep enough bytes in
+//    flight), counting both CTAs' bytes on the leader's barrier
+//    (cta_group::2); one warp of the leader issues every MMA of the pair.
+//    These warps run converged, with one elected lane executing each copy,
+//    MMA and commit, so the operands stay warp-uniform; four softmax
 //    warps per CTA read S from TMEM, apply scale and the ancestor mask, keep
 //    the online softmax (the O rescale is skipped unless the row max grows
 //    by more than 2^8), write bf16 P into shared memory and finally dump O
@@ -56,9 +58,11 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 224;          // 4 softmax + TMA producer + Q loader + MMA warps
+constexpr int kThreads = 256;          // 4 softmax + 2 TMA producers + Q loader + MMA warps
 constexpr int kSoftmaxThreads = 128;
-constexpr int kProdWarp = 4;           // issues the K/V TMA copies of its CTA
+constexpr int kProdWarp = 4;           // warps 4 and 7 issue the K/V TMA copies of their CTA
+constexpr int kProdWarp2 = 7;
+constexpr int kProducers = 2;
 constexpr int kQWarp = 5;
 constexpr int kMmaWarp = 6;            // issues all MMAs; also owns the TMEM allocation
 
@@ -238,11 +242,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 constexpr int kStagesK = kQBlocks;    // 9
 constexpr int kStagesV = 8;
 
-// Warp 4 of each CTA: walks the cluster's stages in order and loads
-// each into the ring with tiled TMA copies from the staging rows. K stage of
-// block kb: box [128 keys x 64 columns] at column 64 kb, keys 128 r .. of the
+// Warps 4 and 7 of each CTA: both walk the cluster's stages in order and
+// each loads every other one into the ring with tiled TMA copies from the
+// staging rows. K stage of block kb: box [128 keys x 64 columns] at column 64 kb, keys 128 r .. of the
 // tile (CTA r). V stage: two boxes [64 keys x 64 columns] at value columns
-// 256 r + 128 h and +64. The leader's thread announces both CTAs' bytes on
+// 256 r + 128 h and +64. The leader's warp announces both CTAs' bytes on
 // its ring_full barrier; the peer's copies count their bytes there too.
 struct Producer {
   const SplitParams& p;
@@ -251,57 +255,59 @@ struct Producer {
   uint32_t rank;
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
+  uint32_t which;      // this warp takes the stages st with st % kProducers == which
   uint32_t st = 0;
+  bool alive = true;
   uint64_t policy = l2_policy_evict_last();   // every K/V tile is re-read by all row tiles
 
-  // Next ring slot: wait until the MMAs of its previous use completed, then
-  // (leader) announce the bytes both CTAs will land on its full barrier.
-  // The whole warp runs this; one elected lane issues each instruction.
+  __device__ bool mine() const { return alive && st % kProducers == which; }
+
+  // The slot of stage st: wait (whole warp) until the MMAs of its previous
+  // use completed, then (leader) announce the bytes both CTAs will land on
+  // its full barrier.
   __device__ bool acquire(uint32_t& dst, uint32_t& bar) {
     const uint32_t stage = st % kNumStages, use = st / kNumStages;
     if (use >= 1) {
       const uint32_t e = smem_addr(&ctrl->ring_empty[stage]), par = (use - 1) & 1u;
       bool ok = false;
       for (int spin = 0; spin < 64 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(e, par));
-      if (!ok && !wait_warp(e, par, ctrl, p, rank)) return false;
+      if (!ok && !wait_warp(e, par, ctrl, p, rank)) return alive = false;
     }
     const uint32_t full = smem_addr(&ctrl->ring_full[stage]);
     if (rank == 0) mbar_arrive_expect_tx_local_elect(full, 2u * kStageBytes);
     bar = map_to_rank(full, 0);
     dst = smem_addr(smem + kOffRing + stage * kStageBytes);
-    ++st;
     return true;
   }
-  __device__ bool load_k(int32_t row0) {
-    for (int kb = 0; kb < kStagesK; ++kb) {
+  __device__ void load_k(int32_t row0) {
+    for (int kb = 0; kb < kStagesK; ++kb, ++st) {
       uint32_t dst, bar;
-      if (!acquire(dst, bar)) return false;
-      tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar, policy);
+      if (mine() && acquire(dst, bar))
+        tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar, policy);
     }
-    return true;
   }
-  __device__ bool load_v(int32_t row0) {
-    for (int v = 0; v < kStagesV; ++v) {
+  __device__ void load_v(int32_t row0) {
+    for (int v = 0; v < kStagesV; ++v, ++st) {
       uint32_t dst, bar;
-      if (!acquire(dst, bar)) return false;
-      const int32_t key = row0 + 64 * (v >> 1);
-      const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
-      tma_load_2d_2sm_elect(dst, tm_v, col, key, bar, policy);
-      tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar, policy);
+      if (mine() && acquire(dst, bar)) {
+        const int32_t key = row0 + 64 * (v >> 1);
+        const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
+        tma_load_2d_2sm_elect(dst, tm_v, col, key, bar, policy);
+        tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar, policy);
+      }
     }
-    return true;
   }
 
   __device__ void run(int64_t u0, int64_t u1) {
     Segment s;
-    for (int64_t u = u0; find_segment(p, u, u1, s); u += s.n) {
+    for (int64_t u = u0; alive && find_segment(p, u, u1, s); u += s.n) {
       const int32_t row0 = (s.kt_base + s.kt0) * kKeysPerTile;
-      if (!load_k(row0)) return;
+      load_k(row0);
       for (int i = 1; i < s.n; ++i) {
-        if (!load_k(row0 + i * kKeysPerTile)) return;
-        if (!load_v(row0 + (i - 1) * kKeysPerTile)) return;
+        load_k(row0 + i * kKeysPerTile);
+        load_v(row0 + (i - 1) * kKeysPerTile);
       }
-      if (!load_v(row0 + (s.n - 1) * kKeysPerTile)) return;
+      load_v(row0 + (s.n - 1) * kKeysPerTile);
     }
   }
 };
@@ -697,8 +703,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
-  } else if (warp == kProdWarp) {
-    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_v};
+  } else if (warp == kProdWarp || warp == kProdWarp2) {
+    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_v, warp == kProdWarp ? 0u : 1u};
     pr.run(u0, u1);
     // After an abort, copies issued before it may still be in flight:
     // give them time to land before the CTA can exit.
