@@ -204,7 +204,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, {"step": f"{rows_per_step} query rows of {rows_total} per step"}),
+        "config": workload_config(wl, {"step": f"{rows_per_step} query rows of {rows_total} per step",
+                                        "l2": "not applicable (float64 oracle on the host cores)"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{rows_per_step} of {rows_total} query rows per step, scaled by rows"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -244,14 +245,18 @@ def run_gpu(args):
     stream = torch.cuda.Stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    # Warm the kernels eagerly once, then capture split and reduce as two graphs.
+    # Warm the kernels eagerly once, then capture the call's three kernels
+    # (KV gather, split, reduce) as three graphs, so that each one's time is
+    # taken with events between them.
     with torch.cuda.stream(stream):
         attn.run(vargs, stream.cuda_stream)
         attn.reduce(vargs, stream.cuda_stream)
     stream.synchronize()
-    g_run, g_red = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_run, stream=stream):
-        attn.run(vargs, stream.cuda_stream)
+    g_gat, g_spl, g_red = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_gat, stream=stream):
+        attn.gather(vargs, stream.cuda_stream)
+    with torch.cuda.graph(g_spl, stream=stream):
+        attn.split(vargs, stream.cuda_stream)
     with torch.cuda.graph(g_red, stream=stream):
         attn.reduce(vargs, stream.cuda_stream)
     code, bits = attn.status(stream.cuda_stream)
@@ -263,16 +268,19 @@ def run_gpu(args):
             flush.zero_()
             if ev is not None:
                 ev[0].record(stream)
-            g_run.replay()
+            g_gat.replay()
             if ev is not None:
                 ev[1].record(stream)
-            g_red.replay()
+            g_spl.replay()
             if ev is not None:
                 ev[2].record(stream)
+            g_red.replay()
+            if ev is not None:
+                ev[3].record(stream)
 
     for _ in range(args.warmup):
         step(None)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_index = int(visible.split(",")[local_rank]) if visible and visible.split(",")[0].isdigit() else local_rank
     with ClockSampler(gpu_index) as clocks:
@@ -288,9 +296,11 @@ def run_gpu(args):
     code, bits = attn.status(stream.cuda_stream)
     if code != 0:
         raise RuntimeError(f"device status {code} ({bits:#x}) after timing")
-    call_ms = [e[0].elapsed_time(e[2]) for e in events]
-    split_ms = [e[0].elapsed_time(e[1]) for e in events]
+    call_ms = [e[0].elapsed_time(e[3]) for e in events]
+    gather_ms = [e[0].elapsed_time(e[1]) for e in events]
+    split_ms = [e[1].elapsed_time(e[2]) for e in events]
     t_call = statistics.mean(call_ms) * 1e-3
+    t_gather = statistics.mean(gather_ms) * 1e-3
     t_split = statistics.mean(split_ms) * 1e-3
 
     # End to end through the public call with host buffers: per step, copy
@@ -324,27 +334,22 @@ def run_gpu(args):
     torch.cuda.synchronize()
     t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
 
-    t_call, t_split, t_e2e = max_over_ranks([t_call, t_split, t_e2e], dist, "cuda")
+    t_call, t_gather, t_split, t_e2e = max_over_ranks([t_call, t_gather, t_split, t_e2e], dist, "cuda")
 
     kv = wl.total_kv
     tflops_split = flops / t_split / 1e12
     t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
-    traffic_path = os.path.join(ROOT, "profiles", "split_kernel_long_traffic.json")
-    traffic = None
-    if os.path.exists(traffic_path):
-        with open(traffic_path) as f:
-            tr = json.load(f)
-        if tr.get("kernel_source_digest") == kernel_digest():
-            traffic = tr.get("dram_bytes_per_launch")
+    traffic = split_traffic()
 
     result = {
         "metric": METRIC, "value": kv * world / t_call, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(wl, {"parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
-                                       "graph": "split and reduce replayed from CUDA graphs"}),
+                                       "graph": "gather, split and reduce replayed from three CUDA graphs"}),
         "detail": {
-            "us_per_call": t_call * 1e6, "split_us": t_split * 1e6, "reduce_us": (t_call - t_split) * 1e6,
+            "us_per_call": t_call * 1e6, "gather_us": t_gather * 1e6, "split_us": t_split * 1e6,
+            "reduce_us": (t_call - t_gather - t_split) * 1e6,
             "kv_tok_per_s_per_gpu": kv / t_call,
             "hbm_gbs_algorithmic": nbytes / t_call / 1e9,
             "tflops_split": tflops_split,
@@ -354,6 +359,7 @@ def run_gpu(args):
         },
         "roofline": {"bound": "tensor", "achieved": tflops_split, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tflops_split / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "verify_split_kernel",
                      "peak_kind": f"{peak_kind} burst bf16 (cuBLAS), kernel timed alone"},
         "clocks": clock_info,
         "e2e": {"value": kv * world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -365,7 +371,7 @@ def run_gpu(args):
         result["cpu_baseline"] = cpu_baseline(inp, oracle.ancestor_masks(inp.parents, inp.qo_indptr))
     if dist is not None:
         dist.barrier()
-        del g_run, g_red
+        del g_gat, g_spl, g_red
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -382,15 +388,36 @@ def max_over_ranks(values, dist, device):
     return [float(x) for x in t.tolist()]
 
 
+SPLIT_SOURCES = ("verify_split_sm100.cu", "sm100_ptx.cuh", "verify_attn_internal.h", "verify_split.h")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_long_traffic.txt")
+
+
 def kernel_digest() -> str:
+    """Digest of the sources that define the split kernel."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_speculative_verify_absorb_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in SPLIT_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
+
+
+def split_traffic():
+    """DRAM bytes per split-kernel launch from the committed ncu summary, or
+    None when the kernel sources changed since that capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    fields = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_source_digest") != kernel_digest():
+        return None
+    return int(fields["dram_bytes_per_launch"])
 
 
 def main():

@@ -160,6 +160,18 @@ int verify_attn_run(const verify_attn_plan_t *plan, const verify_attn_args *args
                     size_t ws_bytes, verify_attn_stream_t stream);
 
 /*
+ * The two halves of verify_attn_run, for callers that time or schedule them
+ * separately: verify_attn_gather copies the referenced latent rows into the
+ * staging rows of ws; verify_attn_split runs the split kernel on them and
+ * must follow a verify_attn_gather with the same plan, args and ws on the
+ * same stream. Same arguments, checks and return codes as verify_attn_run.
+ */
+int verify_attn_gather(const verify_attn_plan_t *plan, const verify_attn_args *args, void *ws,
+                       size_t ws_bytes, verify_attn_stream_t stream);
+int verify_attn_split(const verify_attn_plan_t *plan, const verify_attn_args *args, void *ws,
+                      size_t ws_bytes, verify_attn_stream_t stream);
+
+/*
  * Reduce kernel: LSE-merges every row's partial states from ws into
  * args->out (bf16, round to nearest even), args->lse (natural log) and
  * args->visible_count. Must follow verify_attn_run on the same stream with

@@ -20,9 +20,11 @@ from ._binding import (  # noqa: F401
     verify_attn_build_tree_mask,
     verify_attn_build_tree_mask_device,
     verify_attn_forward_static,
+    verify_attn_gather,
     verify_attn_plan,
     verify_attn_reduce,
     verify_attn_run,
+    verify_attn_split,
     verify_attn_status,
     verify_attn_strerror,
     verify_attn_workspace_init,

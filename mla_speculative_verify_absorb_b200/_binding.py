@@ -64,7 +64,8 @@ _lock = threading.Lock()
 _lib = None
 
 EXPORTS = (
-    "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_reduce",
+    "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_gather", "verify_attn_split",
+    "verify_attn_reduce",
     "verify_attn_build_tree_mask", "verify_attn_build_tree_mask_device", "verify_attn_status",
     "verify_attn_forward_static", "verify_attn_strerror",
 )
@@ -85,6 +86,8 @@ def load_library():
             lib.verify_attn_plan.argtypes = [P(VerifyAttnParams), P(VerifyAttnPlan), P(ctypes.c_size_t)]
             lib.verify_attn_workspace_init.argtypes = [P(VerifyAttnPlan), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_run.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
+            lib.verify_attn_gather.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
+            lib.verify_attn_split.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_reduce.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_build_tree_mask.argtypes = [_vp, _i32, _vp]
             lib.verify_attn_build_tree_mask_device.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp]
@@ -124,6 +127,16 @@ def verify_attn_workspace_init(plan, ws_ptr: int, ws_bytes: int, stream: int = 0
 def verify_attn_run(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stream: int = 0):
     _check(load_library().verify_attn_run(ctypes.byref(plan), ctypes.byref(args), ws_ptr, ws_bytes, stream),
            "verify_attn_run")
+
+
+def verify_attn_gather(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stream: int = 0):
+    _check(load_library().verify_attn_gather(ctypes.byref(plan), ctypes.byref(args), ws_ptr, ws_bytes, stream),
+           "verify_attn_gather")
+
+
+def verify_attn_split(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stream: int = 0):
+    _check(load_library().verify_attn_split(ctypes.byref(plan), ctypes.byref(args), ws_ptr, ws_bytes, stream),
+           "verify_attn_split")
 
 
 def verify_attn_reduce(plan, args: VerifyAttnArgs, ws_ptr: int, ws_bytes: int, stream: int = 0):
@@ -197,6 +210,12 @@ class VerifyAttention:
 
     def run(self, args: VerifyAttnArgs, stream: int):
         verify_attn_run(self.plan, args, _ptr(self.workspace), self.ws_bytes, stream)
+
+    def gather(self, args: VerifyAttnArgs, stream: int):
+        verify_attn_gather(self.plan, args, _ptr(self.workspace), self.ws_bytes, stream)
+
+    def split(self, args: VerifyAttnArgs, stream: int):
+        verify_attn_split(self.plan, args, _ptr(self.workspace), self.ws_bytes, stream)
 
     def reduce(self, args: VerifyAttnArgs, stream: int):
         verify_attn_reduce(self.plan, args, _ptr(self.workspace), self.ws_bytes, stream)

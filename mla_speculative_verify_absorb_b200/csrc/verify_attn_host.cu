@@ -132,11 +132,9 @@ int verify_attn_workspace_init(const verify_attn_plan_t* plan, void* ws, size_t 
   return VERIFY_ATTN_OK;
 }
 
-int verify_attn_run(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws, size_t ws_bytes,
-                    verify_attn_stream_t stream) {
-  int rc = check_args(plan, a, ws, ws_bytes, false);
-  if (rc) return rc;
-  va::SplitParams p;
+namespace {
+
+void fill_split(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws, va::SplitParams& p) {
   p.q_latent = a->q_latent;
   p.ql_tok = a->q_latent_stride_tok;
   p.ql_head = a->q_latent_stride_head;
@@ -163,7 +161,11 @@ int verify_attn_run(const verify_attn_plan_t* plan, const verify_attn_args* a, v
   p.partial = reinterpret_cast<float*>(base + plan->ws_partial_offset);
   p.stage = reinterpret_cast<const uint16_t*>(base + plan->ws_stage_offset);
   p.stage_rows = plan->stage_rows;
+}
 
+cudaError_t launch_gather_for(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws,
+                              cudaStream_t stream) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
   va::GatherParams gp;
   gp.kv_pool = a->kv_pool;
   gp.kv_stride = a->kv_row_stride;
@@ -174,13 +176,48 @@ int verify_attn_run(const verify_attn_plan_t* plan, const verify_attn_args* a, v
   gp.max_tree = plan->max_tree;
   gp.max_kv_per_req = plan->max_kv_per_req;
   gp.pool_slots = plan->pool_slots;
-  gp.status = p.status;
+  gp.status = reinterpret_cast<uint32_t*>(base);
   gp.stage = reinterpret_cast<uint16_t*>(base + plan->ws_stage_offset);
   // A grid of a few CTAs per SM loops over the key tiles of the call.
   const int64_t tiles = plan->stage_rows / va::kKeysPerTile;
   gp.stage_tiles = tiles;
   const int64_t grid = tiles < (int64_t)plan->num_clusters * 8 ? tiles : (int64_t)plan->num_clusters * 8;
-  if (va::launch_gather(gp, (int)grid, (cudaStream_t)stream) != cudaSuccess ||
+  return va::launch_gather(gp, (int)grid, stream);
+}
+
+}  // namespace
+
+int verify_attn_gather(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws, size_t ws_bytes,
+                       verify_attn_stream_t stream) {
+  int rc = check_args(plan, a, ws, ws_bytes, false);
+  if (rc) return rc;
+  if (launch_gather_for(plan, a, ws, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
+int verify_attn_split(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws, size_t ws_bytes,
+                      verify_attn_stream_t stream) {
+  int rc = check_args(plan, a, ws, ws_bytes, false);
+  if (rc) return rc;
+  va::SplitParams p;
+  fill_split(plan, a, ws, p);
+  if (va::launch_split(p, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
+int verify_attn_run(const verify_attn_plan_t* plan, const verify_attn_args* a, void* ws, size_t ws_bytes,
+                    verify_attn_stream_t stream) {
+  int rc = check_args(plan, a, ws, ws_bytes, false);
+  if (rc) return rc;
+  va::SplitParams p;
+  fill_split(plan, a, ws, p);
+  if (launch_gather_for(plan, a, ws, (cudaStream_t)stream) != cudaSuccess ||
       va::launch_split(p, (cudaStream_t)stream) != cudaSuccess) {
     cudaGetLastError();
     return VERIFY_ATTN_CUDA_ERROR;
