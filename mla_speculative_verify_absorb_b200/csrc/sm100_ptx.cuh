@@ -119,6 +119,20 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   return pol;
 }
 
+// Tiled load of one box of a 3-D tensor map at (x, y, z), by one elected
+// lane of a converged warp, bytes counted on `cluster_bar` (cta_group::2),
+// with an L2 cache policy for the loaded lines.
+__device__ __forceinline__ void tma_load_3d_2sm_elect(uint32_t dst, const void* tmap, int32_t x, int32_t y, int32_t z,
+                                                      uint32_t cluster_bar, uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;\n\t}" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(cluster_bar), "l"(policy)
+      : "memory");
+}
+
 // tma_load_2d_2sm by one elected lane of a converged warp, with an L2 cache
 // policy for the loaded lines.
 __device__ __forceinline__ void tma_load_2d_2sm_elect(uint32_t dst, const void* tmap, int32_t x, int32_t y,

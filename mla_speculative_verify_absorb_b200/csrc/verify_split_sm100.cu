@@ -245,8 +245,8 @@ constexpr int kStagesV = 8;
 // Warps 4 and 7 of each CTA: both walk the cluster's stages in order and
 // each loads every other one into the ring with tiled TMA copies from the
 // staging rows. K stage of block kb: box [128 keys x 64 columns] at column 64 kb, keys 128 r .. of the
-// tile (CTA r). V stage: two boxes [64 keys x 64 columns] at value columns
-// 256 r + 128 h and +64. The leader's warp announces both CTAs' bytes on
+// tile (CTA r). V stage: one box of a 3-D view of the same rows, [2 column
+// blocks x 64 keys x 64 columns], value columns 256 r + 128 h .. + 127. The leader's warp announces both CTAs' bytes on
 // its ring_full barrier; the peer's copies count their bytes there too.
 struct Producer {
   const SplitParams& p;
@@ -290,10 +290,9 @@ struct Producer {
     for (int v = 0; v < kStagesV; ++v, ++st) {
       uint32_t dst, bar;
       if (mine() && acquire(dst, bar)) {
+        // One box [2 column blocks][64 keys][64 columns]: blocks 4 r + 2 h, +1.
         const int32_t key = row0 + 64 * (v >> 1);
-        const int32_t col = 256 * (int32_t)rank + 128 * (v & 1);
-        tma_load_2d_2sm_elect(dst, tm_v, col, key, bar, policy);
-        tma_load_2d_2sm_elect(dst + 8192, tm_v, col + 64, key, bar, policy);
+        tma_load_3d_2sm_elect(dst, tm_v, 0, key, 4 * (int32_t)rank + 2 * (v & 1), bar, policy);
       }
     }
   }
@@ -766,6 +765,29 @@ cudaError_t encode_stage_map(const SplitParams& p, uint32_t box_rows, CUtensorMa
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D view of the staging rows for V stages: (64 columns of a block, key row,
+// 64-column block index) with strides (2 B, 1152 B, 128 B); a box [2 blocks x
+// 64 keys x 64 columns] lands as two 8 KB blocks of 64 swizzled 128-byte rows,
+// the MN-major operand layout of the value MMA.
+cudaError_t encode_stage_blocks_map(const SplitParams& p, CUtensorMap* map) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  const cuuint64_t dims[3] = {64, (cuuint64_t)p.stage_rows, (cuuint64_t)(kDQK / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)kDQK * 2, 128};
+  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(p.stage), dims, strides, box,
+                      estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 int split_smem_bytes() { return kSmemBytes; }
@@ -800,7 +822,7 @@ cudaError_t launch_split(const SplitParams& p, cudaStream_t stream) {
   CUtensorMap tm_k, tm_v;
   e = encode_stage_map(p, 128, &tm_k);
   if (e != cudaSuccess) return e;
-  e = encode_stage_map(p, 64, &tm_v);
+  e = encode_stage_blocks_map(p, &tm_v);
   if (e != cudaSuccess) return e;
   verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, tm_k, tm_v);
   return cudaGetLastError();
