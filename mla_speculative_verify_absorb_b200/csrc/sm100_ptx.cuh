@@ -146,6 +146,15 @@ __device__ __forceinline__ void tma_load_2d_2sm_elect(uint32_t dst, const void* 
       : "memory");
 }
 
+// mbar_arrive_local by one elected lane of a converged warp.
+__device__ __forceinline__ void mbar_arrive_local_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
 // mbar_arrive_expect_tx_local by one elected lane of a converged warp.
 __device__ __forceinline__ void mbar_arrive_expect_tx_local_elect(uint32_t bar, uint32_t bytes) {
   asm volatile(

@@ -248,48 +248,70 @@ constexpr int kStagesV = 8;
 // tile (CTA r). V stage: one box of a 3-D view of the same rows, [2 column
 // blocks x 64 keys x 64 columns], value columns 256 r + 128 h .. + 127. The leader's warp announces both CTAs' bytes on
 // its ring_full barrier; the peer's copies count their bytes there too.
+// Two consecutive K blocks of a tile travel as one 32 KB copy when their
+// ring slots are adjacent (no wrap); the producers and the issuer take the
+// same decision from the stage index.
+__device__ __forceinline__ int k_blocks_at(int kb, uint32_t st) {
+  return (kb + 1 < kStagesK && (int)(st % kNumStages) + 1 < kNumStages) ? 2 : 1;
+}
+
 struct Producer {
   const SplitParams& p;
   Ctrl* ctrl;
   uint8_t* smem;
   uint32_t rank;
-  const CUtensorMap* tm_k;
-  const CUtensorMap* tm_v;
-  uint32_t which;      // this warp takes the stages st with st % kProducers == which
-  uint32_t st = 0;
+  const CUtensorMap* tm_k;    // [128 keys x 64 columns] boxes
+  const CUtensorMap* tm_k2;   // [2 blocks x 128 keys x 64 columns] boxes
+  const CUtensorMap* tm_v;    // [2 blocks x 64 keys x 64 columns] boxes
+  uint32_t which;      // this warp takes the copies op with op % kProducers == which
+  uint32_t st = 0, op = 0;
   bool alive = true;
   uint64_t policy = l2_policy_evict_last();   // every K/V tile is re-read by all row tiles
 
-  __device__ bool mine() const { return alive && st % kProducers == which; }
+  __device__ bool mine() const { return alive && op % kProducers == which; }
 
-  // The slot of stage st: wait (whole warp) until the MMAs of its previous
-  // use completed, then (leader) announce the bytes both CTAs will land on
-  // its full barrier.
-  __device__ bool acquire(uint32_t& dst, uint32_t& bar) {
-    const uint32_t stage = st % kNumStages, use = st / kNumStages;
+  // The n (1 or 2) slots of stages st..st+n-1: wait (whole warp) until the
+  // MMAs of the last slot's previous use completed (stages are released in
+  // order, so the earlier slot is free too), then (leader) announce the bytes
+  // both CTAs will land on the first slot's full barrier and complete the
+  // other slot's phase with a plain arrival.
+  __device__ bool acquire(int n, uint32_t& dst, uint32_t& bar) {
+    const uint32_t last = st + (uint32_t)n - 1;
+    const uint32_t use = last / kNumStages;
     if (use >= 1) {
-      const uint32_t e = smem_addr(&ctrl->ring_empty[stage]), par = (use - 1) & 1u;
+      const uint32_t e = smem_addr(&ctrl->ring_empty[last % kNumStages]), par = (use - 1) & 1u;
       bool ok = false;
       for (int spin = 0; spin < 64 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(e, par));
       if (!ok && !wait_warp(e, par, ctrl, p, rank)) return alive = false;
     }
+    const uint32_t stage = st % kNumStages;
     const uint32_t full = smem_addr(&ctrl->ring_full[stage]);
-    if (rank == 0) mbar_arrive_expect_tx_local_elect(full, 2u * kStageBytes);
+    if (rank == 0) {
+      mbar_arrive_expect_tx_local_elect(full, (uint32_t)n * 2u * kStageBytes);
+      if (n == 2) mbar_arrive_local_elect(smem_addr(&ctrl->ring_full[stage + 1]));
+    }
     bar = map_to_rank(full, 0);
     dst = smem_addr(smem + kOffRing + stage * kStageBytes);
     return true;
   }
   __device__ void load_k(int32_t row0) {
-    for (int kb = 0; kb < kStagesK; ++kb, ++st) {
+    for (int kb = 0; kb < kStagesK; ++op) {
+      const int n = k_blocks_at(kb, st);
       uint32_t dst, bar;
-      if (mine() && acquire(dst, bar))
-        tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar, policy);
+      if (mine() && acquire(n, dst, bar)) {
+        if (n == 2)
+          tma_load_3d_2sm_elect(dst, tm_k2, 0, row0 + 128 * (int32_t)rank, kb, bar, policy);
+        else
+          tma_load_2d_2sm_elect(dst, tm_k, 64 * kb, row0 + 128 * (int32_t)rank, bar, policy);
+      }
+      st += (uint32_t)n;
+      kb += n;
     }
   }
   __device__ void load_v(int32_t row0) {
-    for (int v = 0; v < kStagesV; ++v, ++st) {
+    for (int v = 0; v < kStagesV; ++v, ++st, ++op) {
       uint32_t dst, bar;
-      if (mine() && acquire(dst, bar)) {
+      if (mine() && acquire(1, dst, bar)) {
         // One box [2 column blocks][64 keys][64 columns]: blocks 4 r + 2 h, +1.
         const int32_t key = row0 + 64 * (v >> 1);
         tma_load_3d_2sm_elect(dst, tm_v, 0, key, 4 * (int32_t)rank + 2 * (v & 1), bar, policy);
@@ -404,15 +426,20 @@ struct Issuer {
     // S buffer j&1 is free once the softmax warps have read S of tile j-2.
     if (j >= 2 && !wait_bar(&ctrl->s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u)) return false;
     const uint32_t dt = tmem + kColS0 + (uint32_t)(j & 1) * 128;
-    for (int kb = 0; kb < kStagesK; ++kb) {
+    for (int kb0 = 0; kb0 < kStagesK;) {
+      const int n = k_blocks_at(kb0, st);   // a two-block copy lands on its first stage's barrier
       uint32_t saddr;
       if (!wait_stage(saddr)) return false;
-      const uint64_t bd = sdesc_sw128(saddr, 16, 1024);
+      for (int b = 0; b < n; ++b) {
+        const int kb = kb0 + b;
+        const uint64_t bd = sdesc_sw128(saddr + (uint32_t)b * kStageBytes, 16, 1024);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_2sm_bf16_elect(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4), kIdescQK,
-                           (kb | k) != 0);
-      release_stage();
+        for (int k = 0; k < 4; ++k)
+          mma_2sm_bf16_elect(dt, qd + (uint64_t)((kb * 8192 + k * 32) >> 4), bd + (uint64_t)((k * 32) >> 4),
+                             kIdescQK, (kb | k) != 0);
+        release_stage();
+      }
+      kb0 += n;
     }
     if (last_of_segment) commit_both(&ctrl->q_empty);
     commit_both(&ctrl->s_full[j & 1]);
@@ -653,7 +680,7 @@ struct Softmax {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     verify_split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v) {
+                        const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kOffCtrl);
@@ -683,6 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   if (warp == kProdWarp && (threadIdx.x & 31) == 0) {
     prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_k2);
     prefetch_tmap(&tm_v);
   }
   if (warp == kMmaWarp) {
@@ -703,7 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
   } else if (warp == kProdWarp || warp == kProdWarp2) {
-    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_v, warp == kProdWarp ? 0u : 1u};
+    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_k2, &tm_v, warp == kProdWarp ? 0u : 1u};
     pr.run(u0, u1);
     // After an abort, copies issued before it may still be in flight:
     // give them time to land before the CTA can exit.
@@ -765,11 +793,12 @@ cudaError_t encode_stage_map(const SplitParams& p, uint32_t box_rows, CUtensorMa
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// 3-D view of the staging rows for V stages: (64 columns of a block, key row,
-// 64-column block index) with strides (2 B, 1152 B, 128 B); a box [2 blocks x
-// 64 keys x 64 columns] lands as two 8 KB blocks of 64 swizzled 128-byte rows,
-// the MN-major operand layout of the value MMA.
-cudaError_t encode_stage_blocks_map(const SplitParams& p, CUtensorMap* map) {
+// 3-D view of the staging rows: (64 columns of a block, key row, 64-column
+// block index) with strides (2 B, 1152 B, 128 B). A box [2 blocks x 64 keys x
+// 64 columns] lands as two 8 KB blocks of 64 swizzled 128-byte rows (a V
+// stage, the MN-major operand of the value MMA); a box [2 blocks x 128 keys
+// x 64 columns] as two consecutive K stages.
+cudaError_t encode_stage_blocks_map(const SplitParams& p, uint32_t box_keys, CUtensorMap* map) {
   static EncodeTiledFn encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -780,7 +809,7 @@ cudaError_t encode_stage_blocks_map(const SplitParams& p, CUtensorMap* map) {
   }
   const cuuint64_t dims[3] = {64, (cuuint64_t)p.stage_rows, (cuuint64_t)(kDQK / 64)};
   const cuuint64_t strides[2] = {(cuuint64_t)kDQK * 2, 128};
-  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t box[3] = {64, box_keys, 2};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(p.stage), dims, strides, box,
                       estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -819,12 +848,14 @@ cudaError_t split_max_active_clusters(int* n) {
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream) {
   cudaError_t e = configure_split();
   if (e != cudaSuccess) return e;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_k2, tm_v;
   e = encode_stage_map(p, 128, &tm_k);
   if (e != cudaSuccess) return e;
-  e = encode_stage_blocks_map(p, &tm_v);
+  e = encode_stage_blocks_map(p, 128, &tm_k2);
   if (e != cudaSuccess) return e;
-  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, tm_k, tm_v);
+  e = encode_stage_blocks_map(p, 64, &tm_v);
+  if (e != cudaSuccess) return e;
+  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, tm_k, tm_k2, tm_v);
   return cudaGetLastError();
 }
 
