@@ -254,6 +254,10 @@ constexpr int kStagesV = 8;
 __device__ __forceinline__ int k_blocks_at(int kb, uint32_t st) {
   return (kb + 1 < kStagesK && (int)(st % kNumStages) + 1 < kNumStages) ? 2 : 1;
 }
+// Likewise the two V stages of one 64-key quarter (value halves h = 0, 1).
+__device__ __forceinline__ int v_stages_at(int v, uint32_t st) {
+  return ((v & 1) == 0 && (int)(st % kNumStages) + 1 < kNumStages) ? 2 : 1;
+}
 
 struct Producer {
   const SplitParams& p;
@@ -263,6 +267,7 @@ struct Producer {
   const CUtensorMap* tm_k;    // [128 keys x 64 columns] boxes
   const CUtensorMap* tm_k2;   // [2 blocks x 128 keys x 64 columns] boxes
   const CUtensorMap* tm_v;    // [2 blocks x 64 keys x 64 columns] boxes
+  const CUtensorMap* tm_v2;   // [4 blocks x 64 keys x 64 columns] boxes
   uint32_t which;      // this warp takes the copies op with op % kProducers == which
   uint32_t st = 0, op = 0;
   bool alive = true;
@@ -309,13 +314,20 @@ struct Producer {
     }
   }
   __device__ void load_v(int32_t row0) {
-    for (int v = 0; v < kStagesV; ++v, ++st, ++op) {
+    for (int v = 0; v < kStagesV; ++op) {
+      const int n = v_stages_at(v, st);
       uint32_t dst, bar;
-      if (mine() && acquire(1, dst, bar)) {
-        // One box [2 column blocks][64 keys][64 columns]: blocks 4 r + 2 h, +1.
+      if (mine() && acquire(n, dst, bar)) {
+        // Stage (quarter q, half h): blocks 4 r + 2 h, +1 of keys 64 q ..;
+        // a pair of stages is the four blocks 4 r .. 4 r + 3.
         const int32_t key = row0 + 64 * (v >> 1);
-        tma_load_3d_2sm_elect(dst, tm_v, 0, key, 4 * (int32_t)rank + 2 * (v & 1), bar, policy);
+        if (n == 2)
+          tma_load_3d_2sm_elect(dst, tm_v2, 0, key, 4 * (int32_t)rank, bar, policy);
+        else
+          tma_load_3d_2sm_elect(dst, tm_v, 0, key, 4 * (int32_t)rank + 2 * (v & 1), bar, policy);
       }
+      st += (uint32_t)n;
+      v += n;
     }
   }
 
@@ -449,16 +461,20 @@ struct Issuer {
   __device__ bool value(int64_t j, bool first_of_segment, int si) {
     if (!wait_bar(&ctrl->p_full, (uint32_t)(j & 1))) return false;
     if (first_of_segment && si > 0 && !wait_bar(&ctrl->o_free, (si - 1) & 1)) return false;
-    for (int v = 0; v < kStagesV; ++v) {
+    for (int v0 = 0; v0 < kStagesV;) {
+      const int n = v_stages_at(v0, st);   // a two-stage copy lands on its first stage's barrier
       uint32_t saddr;
       if (!wait_stage(saddr)) return false;
-      const int kq = v >> 1, dh = v & 1;
-      const uint64_t bd = sdesc_sw128(saddr, 8192, 1024);
+      for (int b = 0; b < n; ++b) {
+        const int v = v0 + b, kq = v >> 1, dh = v & 1;
+        const uint64_t bd = sdesc_sw128(saddr + (uint32_t)b * kStageBytes, 8192, 1024);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_2sm_bf16_elect(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
-                           bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(first_of_segment && kq == 0 && ks == 0));
-      release_stage();
+        for (int ks = 0; ks < 4; ++ks)
+          mma_2sm_bf16_elect(tmem + kColO + dh * 128, pd + (uint64_t)((kq * 8192 + ks * 32) >> 4),
+                             bd + (uint64_t)((ks * 2048) >> 4), kIdescPV, !(first_of_segment && kq == 0 && ks == 0));
+        release_stage();
+      }
+      v0 += n;
     }
     commit_both(&ctrl->pv_done);
     return true;
@@ -680,7 +696,8 @@ struct Softmax {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     verify_split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v) {
+                        const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_v2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kOffCtrl);
@@ -712,6 +729,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_k2);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_v2);
   }
   if (warp == kMmaWarp) {
     tmem_alloc_2sm(smem_addr(&ctrl->tmem_base), kTmemCols);
@@ -731,7 +749,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Softmax sm(p, ctrl, smem, rank, tmem, cluster);
     sm.run(u0, u1);
   } else if (warp == kProdWarp || warp == kProdWarp2) {
-    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_k2, &tm_v, warp == kProdWarp ? 0u : 1u};
+    Producer pr{p, ctrl, smem, rank, &tm_k, &tm_k2, &tm_v, &tm_v2, warp == kProdWarp ? 0u : 1u};
     pr.run(u0, u1);
     // After an abort, copies issued before it may still be in flight:
     // give them time to land before the CTA can exit.
@@ -796,9 +814,10 @@ cudaError_t encode_stage_map(const SplitParams& p, uint32_t box_rows, CUtensorMa
 // 3-D view of the staging rows: (64 columns of a block, key row, 64-column
 // block index) with strides (2 B, 1152 B, 128 B). A box [2 blocks x 64 keys x
 // 64 columns] lands as two 8 KB blocks of 64 swizzled 128-byte rows (a V
-// stage, the MN-major operand of the value MMA); a box [2 blocks x 128 keys
-// x 64 columns] as two consecutive K stages.
-cudaError_t encode_stage_blocks_map(const SplitParams& p, uint32_t box_keys, CUtensorMap* map) {
+// stage, the MN-major operand of the value MMA), [4 blocks x 64 keys x 64
+// columns] as two consecutive V stages, and [2 blocks x 128 keys x 64
+// columns] as two consecutive K stages.
+cudaError_t encode_stage_blocks_map(const SplitParams& p, uint32_t box_keys, uint32_t box_blocks, CUtensorMap* map) {
   static EncodeTiledFn encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -809,7 +828,7 @@ cudaError_t encode_stage_blocks_map(const SplitParams& p, uint32_t box_keys, CUt
   }
   const cuuint64_t dims[3] = {64, (cuuint64_t)p.stage_rows, (cuuint64_t)(kDQK / 64)};
   const cuuint64_t strides[2] = {(cuuint64_t)kDQK * 2, 128};
-  const cuuint32_t box[3] = {64, box_keys, 2};
+  const cuuint32_t box[3] = {64, box_keys, box_blocks};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(p.stage), dims, strides, box,
                       estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -848,14 +867,16 @@ cudaError_t split_max_active_clusters(int* n) {
 cudaError_t launch_split(const SplitParams& p, cudaStream_t stream) {
   cudaError_t e = configure_split();
   if (e != cudaSuccess) return e;
-  CUtensorMap tm_k, tm_k2, tm_v;
+  CUtensorMap tm_k, tm_k2, tm_v, tm_v2;
   e = encode_stage_map(p, 128, &tm_k);
   if (e != cudaSuccess) return e;
-  e = encode_stage_blocks_map(p, 128, &tm_k2);
+  e = encode_stage_blocks_map(p, 128, 2, &tm_k2);
   if (e != cudaSuccess) return e;
-  e = encode_stage_blocks_map(p, 64, &tm_v);
+  e = encode_stage_blocks_map(p, 64, 2, &tm_v);
   if (e != cudaSuccess) return e;
-  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, tm_k, tm_k2, tm_v);
+  e = encode_stage_blocks_map(p, 64, 4, &tm_v2);
+  if (e != cudaSuccess) return e;
+  verify_split_kernel<<<dim3(2 * p.num_clusters), dim3(kThreads), kSmemBytes, stream>>>(p, tm_k, tm_k2, tm_v, tm_v2);
   return cudaGetLastError();
 }
 
