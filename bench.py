@@ -354,6 +354,7 @@ def run_gpu(args):
             "hbm_gbs_algorithmic": nbytes / t_call / 1e9,
             "tflops_split": tflops_split,
             "roofline_us": t_roof * 1e6, "roofline_frac_call": t_roof / t_call,
+            "split_frac_of_sustained_bf16": tflops_split / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
             "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
             "peaks": {k: v for k, v in peaks.items()}, "peaks_kind": peak_kind,
         },
