@@ -286,7 +286,7 @@ struct Producer {
     if (use >= 1) {
       const uint32_t e = smem_addr(&ctrl->ring_empty[last % kNumStages]), par = (use - 1) & 1u;
       bool ok = false;
-      for (int spin = 0; spin < 64 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(e, par));
+      for (int spin = 0; spin < 1024 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(e, par));
       if (!ok && !wait_warp(e, par, ctrl, p, rank)) return alive = false;
     }
     const uint32_t stage = st % kNumStages;
@@ -422,7 +422,7 @@ struct Issuer {
     const uint32_t stage = st % kNumStages, parity = (st / kNumStages) & 1u;
     const uint32_t bar = smem_addr(&ctrl->ring_full[stage]);
     bool ok = false;
-    for (int spin = 0; spin < 256 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(bar, parity));
+    for (int spin = 0; spin < 4096 && !ok; ++spin) ok = __all_sync(0xffffffffu, mbar_test_wait_cta(bar, parity));
     if (!ok && !wait_warp(bar, parity, ctrl, p, rank)) return false;
     saddr = smem_addr(smem + kOffRing + stage * kStageBytes);
     return true;
