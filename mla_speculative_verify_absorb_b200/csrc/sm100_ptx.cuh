@@ -1,7 +1,8 @@
 // Thin inline-PTX wrappers for the sm_100a features the split kernel uses:
-// mbarriers (local and cluster-remote), cp.async, the tcgen05 tensor-memory
-// allocator, tcgen05.mma / commit / ld / st and their fences, and shared
-// memory matrix descriptors for the UMMA canonical 128-byte-swizzled layouts.
+// mbarriers (local and cluster-remote), tiled TMA tensor copies for CTA pairs
+// with L2 cache policies, cp.async, the tcgen05 tensor-memory allocator,
+// tcgen05.mma / commit / ld / st and their fences, and shared memory matrix
+// descriptors for the UMMA canonical 128-byte-swizzled layouts.
 #pragma once
 
 #include <stdint.h>
@@ -91,25 +92,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
-// Arrive on a (possibly remote) barrier and raise its expected transaction bytes.
-__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar), "r"(bytes)
-               : "memory");
-}
-
 // ---------------------------------------------------------------- TMA
-
-// Tiled load of one box of a 2-D tensor map at (x = column, y = row) into this
-// CTA's shared memory at `dst`. With cta_group::2 the landed bytes are counted
-// on the barrier `cluster_bar`, which may live in the peer CTA of the pair.
-__device__ __forceinline__ void tma_load_2d_2sm(uint32_t dst, const void* tmap, int32_t x, int32_t y,
-                                                uint32_t cluster_bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar)
-      : "memory");
-}
 
 // L2 policy that keeps lines in L2 ahead of normally cached data (for tiles
 // that many CTAs re-read).
@@ -133,8 +116,11 @@ __device__ __forceinline__ void tma_load_3d_2sm_elect(uint32_t dst, const void* 
       : "memory");
 }
 
-// tma_load_2d_2sm by one elected lane of a converged warp, with an L2 cache
-// policy for the loaded lines.
+// Tiled load of one box of a 2-D tensor map at (x = column, y = row) into this
+// CTA's shared memory at `dst`, by one elected lane of a converged warp. With
+// cta_group::2 the landed bytes are counted on the barrier `cluster_bar`,
+// which may live in the peer CTA of the pair; `policy` is the L2 cache policy
+// for the loaded lines.
 __device__ __forceinline__ void tma_load_2d_2sm_elect(uint32_t dst, const void* tmap, int32_t x, int32_t y,
                                                       uint32_t cluster_bar, uint64_t policy) {
   asm volatile(
@@ -146,7 +132,7 @@ __device__ __forceinline__ void tma_load_2d_2sm_elect(uint32_t dst, const void* 
       : "memory");
 }
 
-// mbar_arrive_local by one elected lane of a converged warp.
+// Arrive on a barrier of this CTA, by one elected lane of a converged warp.
 __device__ __forceinline__ void mbar_arrive_local_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
@@ -155,7 +141,8 @@ __device__ __forceinline__ void mbar_arrive_local_elect(uint32_t bar) {
       : "memory");
 }
 
-// mbar_arrive_expect_tx_local by one elected lane of a converged warp.
+// Arrive on a barrier of this CTA and raise its expected transaction bytes, by
+// one elected lane of a converged warp.
 __device__ __forceinline__ void mbar_arrive_expect_tx_local_elect(uint32_t bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
@@ -165,23 +152,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_local_elect(uint32_t bar, 
       : "memory");
 }
 
-// tma_load_2d_2sm with an L2 cache policy for the loaded lines.
-__device__ __forceinline__ void tma_load_2d_2sm(uint32_t dst, const void* tmap, int32_t x, int32_t y,
-                                                uint32_t cluster_bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(cluster_bar), "l"(policy)
-      : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
-}
-
-// Arrive on a barrier of this CTA and raise its expected transaction bytes.
-__device__ __forceinline__ void mbar_arrive_expect_tx_local(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------- cp.async
@@ -192,12 +164,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint3
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-// Arrive on a local barrier once all of this thread's earlier cp.async copies
-// have landed (the arrival is made by the hardware; the thread does not wait).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -226,20 +192,10 @@ __device__ __forceinline__ void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem], issued for the CTA pair (cta_group::2).
-__device__ __forceinline__ void mma_2sm_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same, issued by one elected lane of a converged warp: the whole warp
-// runs the issuing code (so descriptors and addresses stay warp-uniform) and
-// exactly one lane executes the tensor-core instruction.
+// D[tmem] (+)= A[smem] * B[smem] for the CTA pair (cta_group::2), issued by one
+// elected lane of a converged warp: the whole warp runs the issuing code (so
+// descriptors and addresses stay warp-uniform) and exactly one lane executes
+// the tensor-core instruction.
 __device__ __forceinline__ void mma_2sm_bf16_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                    uint32_t accumulate) {
   asm volatile(
@@ -251,6 +207,9 @@ __device__ __forceinline__ void mma_2sm_bf16_elect(uint32_t d_tmem, uint64_t a_d
       : "memory");
 }
 
+// Arrive once on the barrier at this shared offset in every CTA of `mask`
+// when all previously issued tcgen05 operations of the issuing thread
+// complete; issued by one elected lane of a converged warp.
 __device__ __forceinline__ void mma_commit_2sm_mc_elect(uint32_t bar, uint16_t mask) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
@@ -259,15 +218,6 @@ __device__ __forceinline__ void mma_commit_2sm_mc_elect(uint32_t bar, uint16_t m
           bar),
       "h"(mask)
       : "memory");
-}
-
-// Arrive once on the barrier at this shared offset in every CTA of `mask`
-// when all previously issued tcgen05 operations of this thread complete.
-__device__ __forceinline__ void mma_commit_2sm_mc(uint32_t bar, uint16_t mask) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-                   bar),
-               "h"(mask)
-               : "memory");
 }
 
 // 32 lanes x 32 consecutive 32-bit columns (one register per column per thread).

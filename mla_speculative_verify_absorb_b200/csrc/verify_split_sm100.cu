@@ -13,9 +13,10 @@
 //
 // How (B200-specific; the pages' sm_120 kernel is prior art, not the plan):
 //  * The KV rows of the call were first copied, in key order, into a
-//    contiguous staging area (verify_gather.cu), so every K and V tile is a
-//    plain 2-D box of a tensor map and moves with tiled TMA copies: no
-//    load/store-unit work per key and no per-key slot lookups here.
+//    contiguous staging area (verify_gather.cu), so every K and V stage is
+//    a box of a 2-D or 3-D tensor map over those rows and moves with tiled
+//    TMA copies (two adjacent stages with one copy where the ring allows):
+//    no load/store-unit work per key and no per-key slot lookups here.
 //  * A cluster of two CTAs on two SMs shares one 128-row tile: each CTA
 //    holds 64 rows of Q in shared memory and the pair issues
 //    tcgen05.mma.cta_group::2 with M = 128. In that mode a CTA's accumulator
