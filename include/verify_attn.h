@@ -206,7 +206,11 @@ int verify_attn_build_tree_mask_device(const int32_t *parents, const int32_t *qo
  * `stream` and synchronises that stream (not capture-safe; call after the
  * work you want to check). Returns VERIFY_ATTN_OK, VERIFY_ATTN_DEVICE_TIMEOUT,
  * VERIFY_ATTN_DEVICE_BAD_INPUT or VERIFY_ATTN_CUDA_ERROR; *detail_h (may be
- * NULL) receives the raw status bits.
+ * NULL) receives the raw status bits: 1 a bounded wait expired, 2 lengths
+ * outside the plan, 4 a slot outside the pool, 8 a tree mask with a bit at or
+ * beyond T or without its own bit. After an expired wait, words 1-3 of the
+ * workspace (uint32) record the first one: 1, the barrier's byte offset in the
+ * split kernel's control block, and parity | rank << 4 | warp << 8.
  */
 int verify_attn_status(const void *ws, verify_attn_stream_t stream, uint32_t *detail_h);
 
