@@ -401,6 +401,152 @@ def run_gpu(args):
         print(json.dumps(result), flush=True)
 
 
+DEFRAG_METRIC = "KV relocation (Tier 1 defragmentation) GB/s at 65k ctx"
+DEFRAG_SOURCES = ("verify_defrag.cu", "verify_defrag.h", "verify_attn_internal.h")
+DEFRAG_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "defrag_kernel_long_traffic.txt")
+
+
+def run_defrag(args):
+    """``--op defrag``: time the KV relocation kernel on the long workload's
+    slot list. Every step moves all 65,600 positions of the request between
+    two free runs appended to the pool (ping-pong, so each step copies every
+    row); the algorithmic bytes are one read and one write of each 1152-byte
+    latent row plus 8 bytes of index traffic per position."""
+    import torch
+
+    import mla_speculative_verify_absorb_b200 as va
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    wl = WORKLOADS[WORKLOAD]
+    inp = generate(wl)
+    P, N, B = wl.pool_slots, wl.total_kv, wl.batch
+    pool = torch.empty((P + 2 * N, 576), dtype=torch.bfloat16, device="cuda")
+    pool[:P].copy_(torch.from_numpy(inp.kv_pool.view(np.int16)).view(torch.bfloat16))
+    idx = torch.from_numpy(inp.kv_indices.astype(np.int32)).cuda()
+    indptr = torch.from_numpy(inp.kv_indptr.astype(np.int32)).cuda()
+    lens = np.diff(inp.kv_indptr)
+    runs = [torch.from_numpy((base + np.concatenate([[0], np.cumsum(lens)[:-1]])).astype(np.int32)).cuda()
+            for base in (P, P + N)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    nbytes = N * 576 * 2 * 2 + N * 8 + (B + 1) * 4 + B * 4
+    budget = int(lens.max())
+
+    for i in range(args.warmup):
+        with torch.cuda.stream(stream):
+            va.defrag(pool, idx, indptr, runs[i & 1], budget, status=status, stream=stream.cuda_stream)
+    stream.synchronize()
+    # One graph per direction, so the timed region holds device work only.
+    graphs = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+    for k in range(2):
+        with torch.cuda.graph(graphs[k], stream=stream):
+            va.defrag(pool, idx, indptr, runs[k], budget, status=status, stream=stream.cuda_stream)
+
+    def step(i, ev):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            ev[0].record(stream)
+            graphs[i & 1].replay()
+            ev[1].record(stream)
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = int(visible.split(",")[local_rank]) if visible and visible.split(",")[0].isdigit() else local_rank
+    with ClockSampler(gpu_index) as clocks:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            step(args.warmup + i, events[i])
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    clock_info = clocks.summary()
+    t = statistics.mean(e[0].elapsed_time(e[1]) for e in events) * 1e-3
+    if int(status.item()) != 0:
+        raise RuntimeError(f"relocation status {int(status.item()):#x}")
+    # The last step left every position in one of the two runs, in order.
+    last = runs[(args.warmup + args.steps - 1) & 1].item() if B == 1 else None
+    if last is not None and not torch.equal(idx.cpu(), torch.arange(last, last + N, dtype=torch.int32)):
+        raise RuntimeError("relocated indices are not the destination run")
+
+    # End to end: the slot list comes from pinned host memory and the
+    # rewritten one goes back; the pool is the device-resident KV cache.
+    idx_h = idx.cpu().pin_memory()
+    e2e_steps = max(1, min(args.steps, 200))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step(i):
+        with torch.cuda.stream(stream):
+            idx.copy_(idx_h, non_blocking=True)
+            va.defrag(pool, idx, indptr, runs[i & 1], budget, status=status, stream=stream.cuda_stream)
+            idx_h.copy_(idx, non_blocking=True)
+
+    base = args.warmup + args.steps
+    for i in range(3):
+        e2e_step(base + i)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(base + 3 + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
+    t, t_e2e = max_over_ranks([t, t_e2e], dist, "cuda")
+
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / t / 1e9
+    result = {
+        "metric": DEFRAG_METRIC, "value": nbytes * world / t / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "op": "defrag",
+        "config": workload_config(wl, {"moved_positions": N, "budget": budget,
+                                       "step": "every position moves between two free runs appended to the pool",
+                                       "graph": "the relocation launch replayed from a CUDA graph",
+                                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}),
+        "detail": {"us_per_call": t * 1e6, "algorithmic_bytes": nbytes, "roofline_us": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6,
+                   "peaks_kind": peak_kind},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": source_traffic(DEFRAG_TRAFFIC_FILE, DEFRAG_SOURCES),
+                     "kernel": "verify_defrag_kernel", "peak_kind": f"{peak_kind} HBM copy"},
+        "clocks": clock_info,
+        "e2e": {"value": nbytes * world / t_e2e / 1e9, "unit": "GB/s", "h2d_bytes_per_step": N * 4,
+                "d2h_bytes_per_step": N * 4},
+        "gpu_launches": args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle.defrag as odf
+
+        host_pool = pool.view(torch.int16).cpu().numpy().view(np.uint16)
+        host_idx = inp.kv_indices.astype(np.int32)
+        dst = (P + np.concatenate([[0], np.cumsum(lens)[:-1]])).astype(np.int32)
+        cores = 1
+        t0 = time.perf_counter()
+        odf.defrag(host_pool, host_idx, inp.kv_indptr, dst, budget)
+        el = time.perf_counter() - t0
+        result["cpu_baseline"] = {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                  "sample": f"the whole relocation of the {N} positions once ({el:.2f} s, "
+                                            "numpy oracle, pool copies included)"}
+    if dist is not None:
+        dist.barrier()
+        del graphs
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def max_over_ranks(values, dist, device):
     """Element-wise max of a list of floats over all ranks (the job's time)."""
     import torch
@@ -416,13 +562,13 @@ SPLIT_SOURCES = ("verify_split_sm100.cu", "sm100_ptx.cuh", "verify_attn_internal
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_long_traffic.txt")
 
 
-def kernel_digest() -> str:
-    """Digest of the sources that define the split kernel."""
+def kernel_digest(sources=SPLIT_SOURCES) -> str:
+    """Digest of the sources that define a kernel (default: the split kernel)."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_speculative_verify_absorb_b200", "csrc")
-    for name in SPLIT_SOURCES:
+    for name in sources:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -431,15 +577,21 @@ def kernel_digest() -> str:
 def split_traffic():
     """DRAM bytes per split-kernel launch from the committed ncu summary, or
     None when the kernel sources changed since that capture."""
-    if not os.path.exists(TRAFFIC_FILE):
+    return source_traffic(TRAFFIC_FILE, SPLIT_SOURCES)
+
+
+def source_traffic(path, sources):
+    """DRAM bytes per launch recorded in `path`, or None when the sources
+    changed since that capture."""
+    if not os.path.exists(path):
         return None
     fields = {}
-    with open(TRAFFIC_FILE) as f:
+    with open(path) as f:
         for line in f:
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-    if fields.get("kernel_source_digest") != kernel_digest():
+    if fields.get("kernel_source_digest") != kernel_digest(sources):
         return None
     return int(fields["dram_bytes_per_launch"])
 
@@ -451,10 +603,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["verify", "defrag"], default="verify",
+                    help="verify: the attention call (default); defrag: the KV relocation kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.op == "defrag":
+        if args.impl == "reference":
+            ap.error("--op defrag has no reference arm: its line carries the oracle's time as cpu_baseline")
+        run_defrag(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -217,6 +217,38 @@ int verify_attn_status(const void *ws, verify_attn_stream_t stream, uint32_t *de
 /* Static string for a return code. */
 const char *verify_attn_strerror(int code);
 
+/*
+ * KV relocation (Tier 1 defragmentation, the step the pages deferred: live
+ * relocation of a request's fragmented page_size=1 slots into contiguous ones
+ * under a copy budget; page "The Execution Phase", section "Tier 0 KV
+ * Defragmentation"). For request b and n_b = min(N_b, budget), KV position
+ * j < n_b moves to slot dst_begin[b] + j: its 576-wide latent row is copied
+ * there (skipped when already there; row padding beyond 576 is not touched)
+ * and kv_indices[kv_indptr[b] + j] is rewritten. Attention over the result
+ * sees exactly the same rows.
+ *
+ * Caller guarantees (not checked, a violation races): no destination slot is
+ * referenced by any other position of the call, and destination runs of
+ * different requests do not overlap. Checked on the device: each source slot
+ * in [0, pool_slots) (else bit 4 of *status, position skipped) and each run
+ * inside the pool (else bit 2, request skipped). Asynchronous on `stream`,
+ * capture-safe, allocates nothing.
+ */
+typedef struct {
+    uint16_t *kv_pool;          /* bf16 [pool_slots, >=576]; read and written */
+    int64_t kv_row_stride;      /* elements between pool rows, >= 576, multiple of 8 */
+    int64_t pool_slots;
+    int32_t *kv_indices;        /* [sum N_b] slots, rewritten in place */
+    const int32_t *kv_indptr;   /* [batch+1] */
+    const int32_t *dst_begin;   /* [batch] first slot of each request's destination run */
+    int32_t batch;              /* >= 1 */
+    int32_t budget;             /* leading positions of each request to place, >= 0 */
+    int64_t max_total_kv;       /* host bound on sum N_b, sizes the grid (any sum is processed) */
+    uint32_t *status;           /* device word receiving error bits, or NULL */
+} verify_attn_defrag_args;
+
+int verify_attn_defrag(const verify_attn_defrag_args *args, verify_attn_stream_t stream);
+
 /* Size of the library-owned workspace used by verify_attn_forward_static. */
 #define VERIFY_ATTN_STATIC_WS_BYTES (128u << 20)
 

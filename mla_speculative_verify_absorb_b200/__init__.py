@@ -11,14 +11,17 @@ from ._binding import (  # noqa: F401
     VERIFY_ATTN_MAX_TREE,
     VERIFY_ATTN_STATIC_WS_BYTES,
     VerifyAttnArgs,
+    VerifyAttnDefragArgs,
     VerifyAttnError,
     VerifyAttnParams,
     VerifyAttnPlan,
     VerifyAttention,
+    defrag,
     lib_path,
     load_library,
     verify_attn_build_tree_mask,
     verify_attn_build_tree_mask_device,
+    verify_attn_defrag,
     verify_attn_forward_static,
     verify_attn_gather,
     verify_attn_plan,

@@ -54,6 +54,13 @@ class VerifyAttnArgs(ctypes.Structure):
     ]
 
 
+class VerifyAttnDefragArgs(ctypes.Structure):
+    _fields_ = [
+        ("kv_pool", _vp), ("kv_row_stride", _i64), ("pool_slots", _i64), ("kv_indices", _vp), ("kv_indptr", _vp),
+        ("dst_begin", _vp), ("batch", _i32), ("budget", _i32), ("max_total_kv", _i64), ("status", _vp),
+    ]
+
+
 class VerifyAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
@@ -67,7 +74,7 @@ EXPORTS = (
     "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_gather", "verify_attn_split",
     "verify_attn_reduce",
     "verify_attn_build_tree_mask", "verify_attn_build_tree_mask_device", "verify_attn_status",
-    "verify_attn_forward_static", "verify_attn_strerror",
+    "verify_attn_forward_static", "verify_attn_defrag", "verify_attn_strerror",
 )
 
 
@@ -93,6 +100,7 @@ def load_library():
             lib.verify_attn_build_tree_mask_device.argtypes = [_vp, _vp, _i32, _vp, _vp, _vp]
             lib.verify_attn_status.argtypes = [_vp, _vp, P(_u32)]
             lib.verify_attn_forward_static.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, _vp]
+            lib.verify_attn_defrag.argtypes = [P(VerifyAttnDefragArgs), _vp]
             lib.verify_attn_strerror.argtypes = [ctypes.c_int]
             lib.verify_attn_strerror.restype = ctypes.c_char_p
             for name in EXPORTS[:-1]:
@@ -166,6 +174,11 @@ def verify_attn_build_tree_mask_device(parents_ptr: int, qo_indptr_ptr: int, bat
                                                              status_ptr, stream), "verify_attn_build_tree_mask_device")
 
 
+def verify_attn_defrag(args: VerifyAttnDefragArgs, stream: int = 0):
+    """Relocate each request's leading KV positions into its destination run (asynchronous)."""
+    _check(load_library().verify_attn_defrag(ctypes.byref(args), stream), "verify_attn_defrag")
+
+
 def verify_attn_status(ws_ptr: int, stream: int = 0):
     """(code, raw status bits) of a workspace; synchronises `stream`."""
     detail = _u32(0)
@@ -177,6 +190,22 @@ def verify_attn_status(ws_ptr: int, stream: int = 0):
 
 def _ptr(t):
     return None if t is None else int(t.data_ptr())
+
+
+def defrag(kv_pool, kv_indices, kv_indptr, dst_begin, budget: int, status=None, max_total_kv=None, stream=None):
+    """Relocate KV rows with device tensors: kv_pool bf16 [slots, >=576] and kv_indices int32 are
+    rewritten in place; kv_indptr / dst_begin int32; status an optional uint32/int32 device word."""
+    import torch
+
+    s = torch.cuda.current_stream(kv_pool.device).cuda_stream if stream is None else stream
+    args = VerifyAttnDefragArgs(
+        kv_pool=_ptr(kv_pool), kv_row_stride=kv_pool.stride(0), pool_slots=kv_pool.shape[0],
+        kv_indices=_ptr(kv_indices), kv_indptr=_ptr(kv_indptr), dst_begin=_ptr(dst_begin),
+        batch=int(kv_indptr.shape[0]) - 1, budget=int(budget),
+        max_total_kv=int(kv_indices.shape[0]) if max_total_kv is None else int(max_total_kv),
+        status=_ptr(status))
+    verify_attn_defrag(args, s)
+    return args
 
 
 class VerifyAttention:

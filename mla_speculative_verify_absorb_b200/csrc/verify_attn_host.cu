@@ -8,6 +8,7 @@
 #include "verify_attn.h"
 #include "verify_attn_internal.h"
 #include "verify_split.h"
+#include "verify_defrag.h"
 
 namespace {
 
@@ -275,6 +276,29 @@ int verify_attn_build_tree_mask_device(const int32_t* parents, const int32_t* qo
                                        uint64_t* anc, uint32_t* status, verify_attn_stream_t stream) {
   if (!parents || !qo_indptr || !anc || batch < 1) return VERIFY_ATTN_EINVAL;
   if (va::launch_tree_mask(parents, qo_indptr, batch, anc, status, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
+int verify_attn_defrag(const verify_attn_defrag_args* a, verify_attn_stream_t stream) {
+  if (!a || !a->kv_pool || !a->kv_indices || !a->kv_indptr || !a->dst_begin) return VERIFY_ATTN_EINVAL;
+  if (a->batch < 1 || a->budget < 0 || a->pool_slots < 1 || a->pool_slots > INT32_MAX) return VERIFY_ATTN_EINVAL;
+  if (!aligned16(a->kv_pool) || !row_stride_ok(a->kv_row_stride) || a->kv_row_stride < va::kDQK)
+    return VERIFY_ATTN_EINVAL;
+  if (a->max_total_kv < 0 || a->max_total_kv > INT32_MAX) return VERIFY_ATTN_EINVAL;
+  va::DefragParams p;
+  p.kv_pool = a->kv_pool;
+  p.kv_stride = a->kv_row_stride;
+  p.pool_slots = a->pool_slots;
+  p.kv_indices = a->kv_indices;
+  p.kv_indptr = a->kv_indptr;
+  p.dst_begin = a->dst_begin;
+  p.batch = a->batch;
+  p.budget = a->budget;
+  p.status = a->status;
+  if (va::launch_defrag(p, a->max_total_kv, (cudaStream_t)stream) != cudaSuccess) {
     cudaGetLastError();
     return VERIFY_ATTN_CUDA_ERROR;
   }
