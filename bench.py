@@ -547,6 +547,167 @@ def run_defrag(args):
         print(json.dumps(result), flush=True)
 
 
+SV_METRIC = METRIC + " — split-verify variant"
+
+
+def run_split_verify(args):
+    """``--op split-verify``: time the split-verify composition (tree block,
+    dense pass, LSE merge) on the long workload, as one graph per call, and
+    each of its kernels from a second pass of per-kernel graphs."""
+    import torch
+
+    import mla_speculative_verify_absorb_b200 as va
+    from workloads import device as wdev
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    wl = WORKLOADS[WORKLOAD]
+    inp = generate(wl)
+    anc = np.concatenate([va.verify_attn_build_tree_mask(inp.parents[int(inp.qo_indptr[b]):int(inp.qo_indptr[b + 1])])
+                          for b in range(wl.batch)])
+    flops, nbytes = algorithmic_work(inp, anc)
+    self_only = np.concatenate([np.uint64(1) << np.arange(int(t), dtype=np.uint64) for t in wl.tree_sizes])
+    dense_flops, _ = algorithmic_work(inp, self_only)
+    peaks, peak_kind = load_peaks()
+    attn = va.VerifyAttention(max_batch=wl.batch, num_heads=wl.num_heads, max_tree=max(wl.tree_sizes),
+                              max_kv_per_req=max(wl.kv_lens), max_total_kv=wl.total_kv, pool_slots=wl.pool_slots,
+                              sm_scale=wl.sm_scale)
+    d = wdev.to_device(inp, anc)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    pos = wdev.positional(d)
+    with torch.cuda.stream(stream):
+        a_d = attn.split_verify(*pos, lse=d["lse"], stream=stream.cuda_stream)   # allocates the scratch once
+    stream.synchronize()
+    sv = attn._sv
+    tokens = inp.q_latent.shape[0]
+    a_t = attn.make_args(*pos[:7], d["out"], lse=sv["lse_t"][:tokens])
+    g_call, g_tb, g_den, g_spl = (torch.cuda.CUDAGraph() for _ in range(4))
+    with torch.cuda.graph(g_call, stream=stream):
+        attn.split_verify(*pos, lse=d["lse"], stream=stream.cuda_stream)
+    with torch.cuda.graph(g_tb, stream=stream):
+        attn.tree_block(a_t, True, sv["self_anc"].data_ptr(), stream.cuda_stream, out_f32_ptr=sv["o_t"].data_ptr())
+    with torch.cuda.graph(g_den, stream=stream):
+        attn.run(a_d, stream.cuda_stream)
+        attn.reduce(a_d, stream.cuda_stream)
+    with torch.cuda.graph(g_spl, stream=stream):
+        attn.split(a_d, stream.cuda_stream)
+    code, bits = attn.status(stream.cuda_stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits:#x}) after warm-up")
+
+    def timed(graph, ev):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            ev[0].record(stream)
+            graph.replay()
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            g_call.replay()
+    ev = {k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+          for k in ("call", "tb", "dense", "split")}
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = int(visible.split(",")[local_rank]) if visible and visible.split(",")[0].isdigit() else local_rank
+    with ClockSampler(gpu_index) as clocks:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            timed(g_call, ev["call"][i])
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    clock_info = clocks.summary()
+    for i in range(args.steps):
+        timed(g_tb, ev["tb"][i])
+        timed(g_den, ev["dense"][i])
+        timed(g_spl, ev["split"][i])
+    with torch.cuda.stream(stream):
+        g_call.replay()   # leave the call's own result in place
+    torch.cuda.synchronize()
+    code, bits = attn.status(stream.cuda_stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits:#x}) after timing")
+    t = {k: statistics.mean(e[0].elapsed_time(e[1]) for e in v) * 1e-3 for k, v in ev.items()}
+
+    # End to end: this call's inputs from pinned host memory, output and LSE back.
+    host = {k: d[k].cpu().pin_memory() for k in ("q_latent", "q_rope", "kv_indices", "kv_indptr", "qo_indptr",
+                                                   "tree_anc")}
+    out_h = torch.empty_like(d["out"], device="cpu").pin_memory()
+    lse_h = torch.empty_like(d["lse"], device="cpu").pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    e2e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k, x in host.items():
+                d[k].copy_(x, non_blocking=True)
+            attn.split_verify(*pos, lse=d["lse"], stream=stream.cuda_stream)
+            out_h.copy_(d["out"], non_blocking=True)
+            lse_h.copy_(d["lse"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) * 1e-3 / e2e_steps
+    keys = ("call", "tb", "dense", "split")
+    vals = max_over_ranks([t[k] for k in keys] + [t_e2e], dist, "cuda")
+    t = dict(zip(keys, vals[:4]))
+    t_e2e = vals[4]
+
+    kv = wl.total_kv
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    tflops_split = dense_flops / t["split"] / 1e12
+    result = {
+        "metric": SV_METRIC, "value": kv * world / t["call"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t["call"] * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "op": "split-verify",
+        "config": workload_config(wl, {"parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
+                                       "graph": "the composition (tree block, gather, split, reduce, merge) "
+                                                "replayed from one CUDA graph"}),
+        "detail": {
+            "us_per_call": t["call"] * 1e6, "tree_block_us": t["tb"] * 1e6,
+            "dense_pass_us": t["dense"] * 1e6, "split_us": t["split"] * 1e6,
+            "merge_us_by_difference": (t["call"] - t["tb"] - t["dense"]) * 1e6,
+            "roofline_us": t_roof * 1e6, "roofline_frac_call": t_roof / t["call"],
+            "algorithmic_flops": flops, "dense_pass_flops": dense_flops, "algorithmic_bytes": nbytes,
+            "peaks_kind": peak_kind,
+        },
+        "roofline": {"bound": "tensor", "achieved": tflops_split, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tflops_split / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "verify_split_kernel (dense pass: prefix + own key)",
+                     "peak_kind": f"{peak_kind} burst bf16 (cuBLAS), kernel timed alone"},
+        "clocks": clock_info,
+        "e2e": {"value": kv * world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,   # tree block, gather, split, reduce, merge per call
+    }
+    if dist is not None:
+        dist.barrier()
+        del g_call, g_tb, g_den, g_spl
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def max_over_ranks(values, dist, device):
     """Element-wise max of a list of floats over all ranks (the job's time)."""
     import torch
@@ -603,15 +764,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["verify", "defrag"], default="verify",
-                    help="verify: the attention call (default); defrag: the KV relocation kernel")
+    ap.add_argument("--op", choices=["verify", "defrag", "split-verify"], default="verify",
+                    help="verify: the attention call (default); defrag: the KV relocation kernel; "
+                         "split-verify: the variant composed of tree block, dense pass and merge")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.op != "verify" and args.impl == "reference":
+        ap.error(f"--op {args.op} has no reference arm of its own (the oracle arm times --op verify)")
     if args.op == "defrag":
-        if args.impl == "reference":
-            ap.error("--op defrag has no reference arm: its line carries the oracle's time as cpu_baseline")
         run_defrag(args)
+    elif args.op == "split-verify":
+        run_split_verify(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -249,6 +249,65 @@ typedef struct {
 
 int verify_attn_defrag(const verify_attn_defrag_args *args, verify_attn_stream_t stream);
 
+/*
+ * Split-verify variant (page "The Architecture Detective", section "The
+ * Split Verify Design": dense attention over the prefix, a tiny masked
+ * attention over the tree block, and an LSE merge of the two). The fused
+ * path (verify_attn_run + verify_attn_reduce) computes the same result in
+ * one pass; the variant is composed from three calls on one stream:
+ *
+ *   1. verify_attn_tree_block(plan, args_t, 1, self_anc, ...): tree keys that
+ *      are strict ancestors of each node -> args_t->out (o_t), args_t->lse
+ *      (lse_t); writes self_anc[t] = 1 << t and, if given, visible_count;
+ *   2. verify_attn_run + verify_attn_reduce with tree_anc = self_anc: the
+ *      prefix keys plus the node's own key -> (o_p, lse_p);
+ *   3. verify_attn_merge_states: (o_p, lse_p) + (o_t, lse_t) -> out, lse.
+ *
+ * verify_attn_tree_block: same argument struct and checks as
+ * verify_attn_reduce. The tree-block output goes to out_f32 (fp32
+ * [sumT, H, 512] contiguous, 16-byte aligned) when that is non-NULL, else to
+ * args->out (bf16, strides as given). The composition uses fp32 so that the
+ * final output is rounded to bf16 once. args->lse (REQUIRED here) receives the
+ * natural-log LSE of the tree-block key set (-inf and a zero row when the set
+ * is empty).
+ * exclude_self = 0 attends every key of the node's ancestor-or-self mask;
+ * 1 leaves the node's own key to the dense pass. self_anc (device uint64
+ * [sumT]) is optional. args->visible_count, if given, receives
+ * L_b + |tree keys attended| (+1 with exclude_self). Status bits as for the
+ * fused path (2 lengths, 4 slot, 8 tree), in the workspace's status word;
+ * the workspace is otherwise untouched. Asynchronous, capture-safe.
+ */
+int verify_attn_tree_block(const verify_attn_plan_t *plan, const verify_attn_args *args, int exclude_self,
+                           uint64_t *self_anc, float *out_f32, void *workspace, size_t workspace_bytes,
+                           verify_attn_stream_t stream);
+
+/*
+ * Two-state LSE merge. Rows are (token, head) with token < min(max_tokens,
+ * *num_tokens) (num_tokens may be NULL: max_tokens rows). o_a, out: bf16
+ * [tokens, H, 512]; o_b: bf16, or fp32 when o_b_f32 = 1; all with the given
+ * strides in elements (multiples of 8, 16-byte aligned bases); lse_a, lse_b,
+ * lse: fp32 [tokens, H] contiguous,
+ * natural log. out may alias o_a or o_b; lse may be NULL. A state with
+ * lse = -inf has weight 0; two such states give a zero row and -inf.
+ */
+typedef struct {
+    const uint16_t *o_a;
+    int64_t o_a_stride_tok, o_a_stride_head;
+    const float *lse_a;
+    const void *o_b;
+    int64_t o_b_stride_tok, o_b_stride_head;
+    const float *lse_b;
+    int32_t o_b_f32;             /* 0: o_b is bf16, 1: fp32 */
+    uint16_t *out;
+    int64_t out_stride_tok, out_stride_head;
+    float *lse;
+    int64_t max_tokens;
+    const int32_t *num_tokens;   /* device int32, or NULL */
+    int32_t num_heads;
+} verify_attn_merge_args;
+
+int verify_attn_merge_states(const verify_attn_merge_args *args, verify_attn_stream_t stream);
+
 /* Size of the library-owned workspace used by verify_attn_forward_static. */
 #define VERIFY_ATTN_STATIC_WS_BYTES (128u << 20)
 

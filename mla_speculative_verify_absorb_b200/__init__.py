@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     VERIFY_ATTN_STATIC_WS_BYTES,
     VerifyAttnArgs,
     VerifyAttnDefragArgs,
+    VerifyAttnMergeArgs,
     VerifyAttnError,
     VerifyAttnParams,
     VerifyAttnPlan,
@@ -24,11 +25,13 @@ from ._binding import (  # noqa: F401
     verify_attn_defrag,
     verify_attn_forward_static,
     verify_attn_gather,
+    verify_attn_merge_states,
     verify_attn_plan,
     verify_attn_reduce,
     verify_attn_run,
     verify_attn_split,
     verify_attn_status,
     verify_attn_strerror,
+    verify_attn_tree_block,
     verify_attn_workspace_init,
 )

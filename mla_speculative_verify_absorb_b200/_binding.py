@@ -61,6 +61,15 @@ class VerifyAttnDefragArgs(ctypes.Structure):
     ]
 
 
+class VerifyAttnMergeArgs(ctypes.Structure):
+    _fields_ = [
+        ("o_a", _vp), ("o_a_stride_tok", _i64), ("o_a_stride_head", _i64), ("lse_a", _vp),
+        ("o_b", _vp), ("o_b_stride_tok", _i64), ("o_b_stride_head", _i64), ("lse_b", _vp), ("o_b_f32", _i32),
+        ("out", _vp), ("out_stride_tok", _i64), ("out_stride_head", _i64), ("lse", _vp),
+        ("max_tokens", _i64), ("num_tokens", _vp), ("num_heads", _i32),
+    ]
+
+
 class VerifyAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
@@ -74,7 +83,8 @@ EXPORTS = (
     "verify_attn_plan", "verify_attn_workspace_init", "verify_attn_run", "verify_attn_gather", "verify_attn_split",
     "verify_attn_reduce",
     "verify_attn_build_tree_mask", "verify_attn_build_tree_mask_device", "verify_attn_status",
-    "verify_attn_forward_static", "verify_attn_defrag", "verify_attn_strerror",
+    "verify_attn_forward_static", "verify_attn_defrag", "verify_attn_tree_block", "verify_attn_merge_states",
+    "verify_attn_strerror",
 )
 
 
@@ -101,6 +111,9 @@ def load_library():
             lib.verify_attn_status.argtypes = [_vp, _vp, P(_u32)]
             lib.verify_attn_forward_static.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), _vp, _vp]
             lib.verify_attn_defrag.argtypes = [P(VerifyAttnDefragArgs), _vp]
+            lib.verify_attn_tree_block.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), ctypes.c_int, _vp, _vp,
+                                                   _vp, ctypes.c_size_t, _vp]
+            lib.verify_attn_merge_states.argtypes = [P(VerifyAttnMergeArgs), _vp]
             lib.verify_attn_strerror.argtypes = [ctypes.c_int]
             lib.verify_attn_strerror.restype = ctypes.c_char_p
             for name in EXPORTS[:-1]:
@@ -177,6 +190,19 @@ def verify_attn_build_tree_mask_device(parents_ptr: int, qo_indptr_ptr: int, bat
 def verify_attn_defrag(args: VerifyAttnDefragArgs, stream: int = 0):
     """Relocate each request's leading KV positions into its destination run (asynchronous)."""
     _check(load_library().verify_attn_defrag(ctypes.byref(args), stream), "verify_attn_defrag")
+
+
+def verify_attn_tree_block(plan, args: VerifyAttnArgs, exclude_self: bool, self_anc_ptr, out_f32_ptr, ws_ptr: int,
+                           ws_bytes: int, stream: int = 0):
+    """Masked tree-block attention of the split-verify variant (asynchronous)."""
+    _check(load_library().verify_attn_tree_block(ctypes.byref(plan), ctypes.byref(args), int(bool(exclude_self)),
+                                                 self_anc_ptr, out_f32_ptr, ws_ptr, ws_bytes, stream),
+           "verify_attn_tree_block")
+
+
+def verify_attn_merge_states(args: VerifyAttnMergeArgs, stream: int = 0):
+    """Two-state LSE merge (asynchronous)."""
+    _check(load_library().verify_attn_merge_states(ctypes.byref(args), stream), "verify_attn_merge_states")
 
 
 def verify_attn_status(ws_ptr: int, stream: int = 0):
@@ -257,6 +283,49 @@ class VerifyAttention:
         self.run(args, s)
         self.reduce(args, s)
         return args
+
+    def tree_block(self, args: VerifyAttnArgs, exclude_self: bool, self_anc_ptr, stream: int, out_f32_ptr=None):
+        verify_attn_tree_block(self.plan, args, exclude_self, self_anc_ptr, out_f32_ptr, _ptr(self.workspace),
+                               self.ws_bytes, stream)
+
+    def split_verify(self, q_latent, q_rope, kv_pool, kv_indices, kv_indptr, qo_indptr, tree_anc, out,
+                     lse=None, visible_count=None, stream=None):
+        """The split-verify variant: tree block (strict ancestors), dense pass
+        (prefix + own key) and LSE merge, three library calls on one stream.
+        Same inputs and results as ``__call__`` (up to rounding). Scratch for
+        the intermediate states is allocated once, sized by the plan."""
+        import torch
+
+        s = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+        tokens = int(q_latent.shape[0])
+        H = self.params.num_heads
+        if getattr(self, "_sv", None) is None:
+            cap = self.params.max_batch * self.params.max_tree
+            self._sv = {
+                "o_t": torch.empty((cap, H, VERIFY_ATTN_D_LATENT), dtype=torch.float32, device=self.device),
+                "lse_t": torch.empty((cap, H), dtype=torch.float32, device=self.device),
+                "lse_p": torch.empty((cap, H), dtype=torch.float32, device=self.device),
+                "self_anc": torch.empty((cap,), dtype=torch.int64, device=self.device),
+            }
+        sv = self._sv
+        if tokens > sv["self_anc"].shape[0]:
+            raise VerifyAttnError(-1, "split_verify: more tokens than the plan allows")
+        o_t, lse_t, lse_p, self_anc = sv["o_t"][:tokens], sv["lse_t"][:tokens], sv["lse_p"][:tokens], sv["self_anc"]
+        a_t = self.make_args(q_latent, q_rope, kv_pool, kv_indices, kv_indptr, qo_indptr, tree_anc, out,
+                             lse=lse_t, visible_count=visible_count)
+        self.tree_block(a_t, True, _ptr(self_anc), s, out_f32_ptr=_ptr(o_t))
+        a_d = self.make_args(q_latent, q_rope, kv_pool, kv_indices, kv_indptr, qo_indptr, self_anc[:tokens], out,
+                             lse=lse_p)
+        self.run(a_d, s)
+        self.reduce(a_d, s)
+        batch = int(kv_indptr.shape[0]) - 1
+        m = VerifyAttnMergeArgs(
+            o_a=_ptr(out), o_a_stride_tok=out.stride(0), o_a_stride_head=out.stride(1), lse_a=_ptr(lse_p),
+            o_b=_ptr(o_t), o_b_stride_tok=o_t.stride(0), o_b_stride_head=o_t.stride(1), lse_b=_ptr(lse_t), o_b_f32=1,
+            out=_ptr(out), out_stride_tok=out.stride(0), out_stride_head=out.stride(1), lse=_ptr(lse),
+            max_tokens=tokens, num_tokens=_ptr(qo_indptr) + 4 * batch, num_heads=H)
+        verify_attn_merge_states(m, s)
+        return a_d
 
     def status(self, stream=None):
         import torch

@@ -9,6 +9,7 @@
 #include "verify_attn_internal.h"
 #include "verify_split.h"
 #include "verify_defrag.h"
+#include "verify_variant.h"
 
 namespace {
 
@@ -276,6 +277,80 @@ int verify_attn_build_tree_mask_device(const int32_t* parents, const int32_t* qo
                                        uint64_t* anc, uint32_t* status, verify_attn_stream_t stream) {
   if (!parents || !qo_indptr || !anc || batch < 1) return VERIFY_ATTN_EINVAL;
   if (va::launch_tree_mask(parents, qo_indptr, batch, anc, status, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
+int verify_attn_tree_block(const verify_attn_plan_t* plan, const verify_attn_args* a, int exclude_self,
+                           uint64_t* self_anc, float* out_f32, void* ws, size_t ws_bytes,
+                           verify_attn_stream_t stream) {
+  int rc = check_args(plan, a, ws, ws_bytes, out_f32 == nullptr);
+  if (rc) return rc;
+  if (!a->lse || (out_f32 && !aligned16(out_f32))) return VERIFY_ATTN_EINVAL;
+  va::TreeBlockParams p;
+  p.q_latent = a->q_latent;
+  p.ql_tok = a->q_latent_stride_tok;
+  p.ql_head = a->q_latent_stride_head;
+  p.q_rope = a->q_rope;
+  p.qr_tok = a->q_rope_stride_tok;
+  p.qr_head = a->q_rope_stride_head;
+  p.kv_pool = a->kv_pool;
+  p.kv_stride = a->kv_row_stride;
+  p.kv_indices = a->kv_indices;
+  p.kv_indptr = a->kv_indptr;
+  p.qo_indptr = a->qo_indptr;
+  p.tree_anc = a->tree_anc;
+  p.batch = a->batch;
+  p.num_heads = plan->num_heads;
+  p.max_tree = plan->max_tree;
+  p.max_kv_per_req = plan->max_kv_per_req;
+  p.pool_slots = plan->pool_slots;
+  p.scale_log2 = plan->sm_scale * 1.4426950408889634f;
+  p.exclude_self = exclude_self ? 1 : 0;
+  p.out = a->out;
+  p.out_f32 = out_f32;
+  p.out_tok = a->out_stride_tok;
+  p.out_head = a->out_stride_head;
+  p.lse = a->lse;
+  p.self_anc = self_anc;
+  p.visible_count = a->visible_count;
+  p.status = static_cast<uint32_t*>(ws);
+  const int64_t max_tokens = (int64_t)plan->max_batch * plan->max_tree;
+  if (va::launch_tree_block(p, max_tokens, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
+int verify_attn_merge_states(const verify_attn_merge_args* a, verify_attn_stream_t stream) {
+  if (!a || !a->o_a || !a->o_b || !a->out || !a->lse_a || !a->lse_b) return VERIFY_ATTN_EINVAL;
+  if (a->num_heads < 1 || a->num_heads > VERIFY_ATTN_MAX_HEADS || a->max_tokens < 0) return VERIFY_ATTN_EINVAL;
+  if (!aligned16(a->o_a) || !aligned16(a->o_b) || !aligned16(a->out)) return VERIFY_ATTN_EINVAL;
+  if (!row_stride_ok(a->o_a_stride_tok) || !row_stride_ok(a->o_a_stride_head) || !row_stride_ok(a->o_b_stride_tok) ||
+      !row_stride_ok(a->o_b_stride_head) || !row_stride_ok(a->out_stride_tok) || !row_stride_ok(a->out_stride_head))
+    return VERIFY_ATTN_EINVAL;
+  va::MergeParams p;
+  p.o_a = a->o_a;
+  p.a_tok = a->o_a_stride_tok;
+  p.a_head = a->o_a_stride_head;
+  p.lse_a = a->lse_a;
+  p.o_b = a->o_b;
+  p.b_tok = a->o_b_stride_tok;
+  p.b_head = a->o_b_stride_head;
+  p.lse_b = a->lse_b;
+  p.b_f32 = a->o_b_f32 ? 1 : 0;
+  p.out = a->out;
+  p.out_tok = a->out_stride_tok;
+  p.out_head = a->out_stride_head;
+  p.lse = a->lse;
+  p.max_tokens = a->max_tokens;
+  p.num_tokens = a->num_tokens;
+  p.num_heads = a->num_heads;
+  if (a->max_tokens == 0) return VERIFY_ATTN_OK;
+  if (va::launch_merge(p, (cudaStream_t)stream) != cudaSuccess) {
     cudaGetLastError();
     return VERIFY_ATTN_CUDA_ERROR;
   }
