@@ -693,8 +693,9 @@ def run_split_verify(args):
             "peaks_kind": peak_kind,
         },
         "roofline": {"bound": "tensor", "achieved": tflops_split, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": tflops_split / peaks["bf16_tflops"], "traffic": None,
-                     "kernel": "verify_split_kernel (dense pass: prefix + own key)",
+                     "frac": tflops_split / peaks["bf16_tflops"], "traffic": split_traffic(),
+                     "kernel": "verify_split_kernel (dense pass: prefix + own key; same kernel and data "
+                               "movement as the fused call, only the mask words differ)",
                      "peak_kind": f"{peak_kind} burst bf16 (cuBLAS), kernel timed alone"},
         "clocks": clock_info,
         "e2e": {"value": kv * world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -10,9 +10,9 @@
 // that the merge rounds to bf16 once, or bf16) and the natural-log LSE of
 // that key set.
 //
-// One CTA per tree token (grid-stride): it gathers the token's visible tree
-// rows (at most 64 x 1152 B) into shared memory once, then each of the eight
-// warps takes every eighth head. A warp holds the 576-wide query in
+// One CTA per (tree token, group of eight heads), grid-stride: it gathers the
+// token's visible tree rows (at most 64 x 1152 B) into shared memory, and
+// each of its eight warps takes one head. A warp holds the 576-wide query in
 // registers (lane l: bf16 pairs l, l+32, ...), forms each score with a warp
 // sum, keeps the scores of keys l and l+32 in lane l, and accumulates the
 // 512-wide output in fp32 (lane l: pairs l, l+32, ..., l+224). The work is a
@@ -56,7 +56,11 @@ __global__ void __launch_bounds__(kTbWarps * 32) verify_tree_block_kernel(const 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int32_t total = p.qo_indptr[p.batch];
 
-  for (int32_t g = blockIdx.x; g < total; g += gridDim.x) {
+  const int head_groups = (p.num_heads + kTbWarps - 1) / kTbWarps;
+  const int64_t items = (int64_t)total * head_groups;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int32_t g = (int32_t)(it / head_groups);
+    const int hg = (int)(it % head_groups);
     int lo = 0, hi = p.batch;   // request b with qo_indptr[b] <= g < qo_indptr[b + 1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(kTbWarps * 32) verify_tree_block_kernel(const 
     }
     const Request r = load_request(p.qo_indptr, p.kv_indptr, lo, 1, p.max_tree, p.max_kv_per_req);
     if (!r.valid) {   // uniform across the CTA
-      if (threadIdx.x == 0) atomicOr(p.status, kStatusBadLengths);
+      if (threadIdx.x == 0 && hg == 0) atomicOr(p.status, kStatusBadLengths);
       continue;
     }
     const int t = g - r.q_begin;
@@ -75,7 +79,7 @@ __global__ void __launch_bounds__(kTbWarps * 32) verify_tree_block_kernel(const 
     uint64_t bits = anc & in_tree;
     if (p.exclude_self) bits &= ~self;
     const int n = __popcll(bits);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && hg == 0) {
       if ((anc & ~in_tree) != 0ull || (anc & self) == 0ull) atomicOr(p.status, kStatusBadTree);
       if (p.self_anc) p.self_anc[g] = self;
       if (p.visible_count) p.visible_count[g] = (int32_t)(L + n + (p.exclude_self ? 1 : 0));
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(kTbWarps * 32) verify_tree_block_kernel(const 
     for (int k = warp; k < n; k += kTbWarps) {
       const int32_t slot = p.kv_indices[r.kv_begin + L + s_key[k]];
       const bool ok = slot >= 0 && (int64_t)slot < p.pool_slots;
-      if (!ok && lane == 0) atomicOr(p.status, kStatusBadSlot);
+      if (!ok && lane == 0 && hg == 0) atomicOr(p.status, kStatusBadSlot);
       const int4* src = reinterpret_cast<const int4*>(p.kv_pool + (int64_t)(ok ? slot : 0) * p.kv_stride);
       int4* dst = reinterpret_cast<int4*>(tb_smem + (size_t)k * kDQK * 2);
 #pragma unroll
@@ -99,7 +103,8 @@ __global__ void __launch_bounds__(kTbWarps * 32) verify_tree_block_kernel(const 
     }
     __syncthreads();
 
-    for (int h = warp; h < p.num_heads; h += kTbWarps) {
+    const int h = hg * kTbWarps + warp;
+    if (h < p.num_heads) {
       const uint32_t* ql = reinterpret_cast<const uint32_t*>(p.q_latent + (int64_t)g * p.ql_tok + (int64_t)h * p.ql_head);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(p.q_rope + (int64_t)g * p.qr_tok + (int64_t)h * p.qr_head);
       float2 q[9];
@@ -173,7 +178,8 @@ cudaError_t launch_tree_block(const TreeBlockParams& p, int64_t max_tokens, cuda
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = 1;
   }
-  int64_t grid = max_tokens < 148 * 2 ? max_tokens : 148 * 2;
+  const int64_t items = max_tokens * ((p.num_heads + kTbWarps - 1) / kTbWarps);
+  int64_t grid = items < 148 * 4 ? items : 148 * 4;
   if (grid < 1) grid = 1;
   verify_tree_block_kernel<<<(unsigned)grid, kTbWarps * 32, kTbSmem, stream>>>(p);
   return cudaGetLastError();
