@@ -709,6 +709,176 @@ def run_split_verify(args):
         print(json.dumps(result), flush=True)
 
 
+SHARD_METRIC = METRIC + " — KV-sequence sharded"
+
+
+def run_sequence_shard(args):
+    """``--op sequence-shard``: the long call with its KV split over the N
+    ranks (strong scaling: one request, fixed total work). Each rank attends
+    its shard, the states are all-gathered over NCCL and every rank merges
+    them; the time is the max over ranks of that whole sequence. With one
+    GPU the same line also reports, for R = 2, 4, 8, each shard's pass and
+    the stacked merge run one after another on this GPU (what a rank
+    computes; the exchange is not part of those figures)."""
+    import torch
+
+    import mla_speculative_verify_absorb_b200 as va
+    from mla_speculative_verify_absorb_b200.sequence_shard import ShardedVerify
+    from workloads import device as wdev
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    wl = WORKLOADS[WORKLOAD]
+    inp = generate(wl)
+    anc = np.concatenate([va.verify_attn_build_tree_mask(inp.parents[int(inp.qo_indptr[b]):int(inp.qo_indptr[b + 1])])
+                          for b in range(wl.batch)])
+    flops, nbytes = algorithmic_work(inp, anc)
+    peaks, peak_kind = load_peaks()
+    d = wdev.to_device(inp, anc)
+    T, L, H = int(wl.tree_sizes[0]), int(wl.prefixes[0]), wl.num_heads
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    s = stream.cuda_stream
+
+    def make(R):
+        return ShardedVerify(world=R, num_heads=H, max_tree=T, max_prefix=L, pool_slots=wl.pool_slots,
+                             sm_scale=wl.sm_scale)
+
+    def local(sv, r, o, lse):
+        return sv.local_state(r, d["q_latent"], d["q_rope"], d["kv_pool"], d["kv_indices"], d["tree_anc"], o, lse, s)
+
+    def timed_graph(g, reps):
+        ts = []
+        for _ in range(reps):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                e[0].record(stream)
+                g.replay()
+                e[1].record(stream)
+            ts.append(e)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ts) * 1e-3
+
+    sv = make(world)
+    if dist is not None:
+        with torch.cuda.stream(stream):
+            sv(d["q_latent"], d["q_rope"], d["kv_pool"], d["kv_indices"], d["tree_anc"], d["out"], d["lse"],
+               stream=s)
+    else:
+        o_all, lse_all = sv.stacked(T)
+        g_call = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            local(sv, 0, o_all[0], lse_all[0])
+            sv.merge(o_all, lse_all, d["out"], d["lse"], s)
+        stream.synchronize()
+        with torch.cuda.graph(g_call, stream=stream):
+            local(sv, 0, o_all[0], lse_all[0])
+            sv.merge(o_all, lse_all, d["out"], d["lse"], s)
+
+    def call():
+        with torch.cuda.stream(stream):
+            if dist is None:
+                g_call.replay()
+            else:
+                sv(d["q_latent"], d["q_rope"], d["kv_pool"], d["kv_indices"], d["tree_anc"], d["out"], d["lse"],
+                   stream=s)
+
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+        call()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = int(visible.split(",")[local_rank]) if visible and visible.split(",")[0].isdigit() else local_rank
+    with ClockSampler(gpu_index) as clocks:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                events[i][0].record(stream)
+            call()
+            with torch.cuda.stream(stream):
+                events[i][1].record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    clock_info = clocks.summary()
+    t_call = statistics.mean(a.elapsed_time(b) for a, b in events) * 1e-3
+    code, bits = sv.attn.status(s)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({bits:#x})")
+
+    emulated = {}
+    if dist is None:
+        reps = max(3, min(args.steps, 100))
+        for R in (2, 4, 8):
+            svR = make(R)
+            o_all, lse_all = svR.stacked(T)
+            shard_t = []
+            for r in range(R):
+                with torch.cuda.stream(stream):
+                    ok = local(svR, r, o_all[r], lse_all[r])
+                stream.synchronize()
+                if not ok:
+                    raise RuntimeError("every shard of the long call has keys")
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    local(svR, r, o_all[r], lse_all[r])
+                shard_t.append(timed_graph(g, reps))
+            gm = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                svR.merge(o_all, lse_all, d["out"], d["lse"], s)
+            stream.synchronize()
+            with torch.cuda.graph(gm, stream=stream):
+                svR.merge(o_all, lse_all, d["out"], d["lse"], s)
+            t_merge = timed_graph(gm, reps)
+            code, bits = svR.attn.status(s)
+            if code != 0:
+                raise RuntimeError(f"device status {code} ({bits:#x}) at R={R}")
+            emulated[str(R)] = {"max_shard_us": max(shard_t) * 1e6, "min_shard_us": min(shard_t) * 1e6,
+                                "merge_us": t_merge * 1e6,
+                                "exchange_bytes_per_rank_out": T * H * (512 * 2 + 4),
+                                "exchange_bytes_per_rank_in": (R - 1) * T * H * (512 * 2 + 4)}
+    (t_call,) = max_over_ranks([t_call], dist, "cuda")
+    kv = wl.total_kv
+    t_roof = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    achieved = flops / t_call / 1e12
+    result = {
+        "metric": SHARD_METRIC, "value": kv / t_call, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "op": "sequence-shard",
+        "config": workload_config(wl, {"parallelism": f"KV sequence split over {world} ranks, NCCL all-gather of "
+                                                      "(o, lse), stacked LSE merge" if world > 1 else
+                                                      "1 GPU (one shard, merge of one state)"}),
+        "detail": {"us_per_call": t_call * 1e6, "roofline_us": t_roof * 1e6, "roofline_frac_call": t_roof / t_call,
+                   "emulated_ranks_on_one_gpu": emulated, "algorithmic_flops": flops,
+                   "algorithmic_bytes": nbytes, "peaks_kind": peak_kind},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "whole sharded call (gather, split, reduce, merge; all-gather when N > 1)",
+                     "peak_kind": f"{peak_kind} burst bf16 (cuBLAS)"},
+        "clocks": clock_info,
+        "gpu_launches": 4 * args.steps,   # gather, split, reduce, merge per call (plus NCCL when N > 1)
+    }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def max_over_ranks(values, dist, device):
     """Element-wise max of a list of floats over all ranks (the job's time)."""
     import torch
@@ -765,9 +935,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["verify", "defrag", "split-verify"], default="verify",
+    ap.add_argument("--op", choices=["verify", "defrag", "split-verify", "sequence-shard"], default="verify",
                     help="verify: the attention call (default); defrag: the KV relocation kernel; "
-                         "split-verify: the variant composed of tree block, dense pass and merge")
+                         "split-verify: the variant composed of tree block, dense pass and merge; "
+                         "sequence-shard: the call with its KV split over the ranks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -777,6 +948,8 @@ def main():
         run_defrag(args)
     elif args.op == "split-verify":
         run_split_verify(args)
+    elif args.op == "sequence-shard":
+        run_sequence_shard(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -308,6 +308,36 @@ typedef struct {
 
 int verify_attn_merge_states(const verify_attn_merge_args *args, verify_attn_stream_t stream);
 
+/*
+ * Stacked R-state LSE merge, the combine step of KV-sequence sharding: each
+ * of R ranks attends a disjoint part of every row's visible keys (its
+ * prefix chunk; the last rank also takes the tree block) and returns
+ * (o_r, lse_r); the R states are gathered along a leading axis and merged
+ * (page "The Breakthrough", section "The Message in Context": KV-split
+ * partials combined by a reduce; page "The Architecture Detective",
+ * section "The Split Verify Design": LSE merge). With m = max_r lse_r and
+ * w_r = exp(lse_r - m): out = sum_r w_r o_r / sum_r w_r, lse = m + ln sum_r w_r.
+ * States with lse = -inf have weight 0; all empty gives a zero row and -inf.
+ *
+ * o: bf16 [R, max_tokens, H, 512] contiguous, 16-byte aligned; lse_states:
+ * fp32 [R, max_tokens, H]; out: bf16 [tokens, H, 512] with the given strides
+ * (multiples of 8 elements); lse: fp32 [tokens, H] or NULL. Rows are tokens <
+ * min(max_tokens, *num_tokens) (num_tokens may be NULL). out must not alias o.
+ */
+typedef struct {
+    const uint16_t *o;
+    const float *lse_states;
+    int32_t num_states;          /* R, 1..1024 */
+    int32_t num_heads;
+    uint16_t *out;
+    int64_t out_stride_tok, out_stride_head;
+    float *lse;
+    int64_t max_tokens;
+    const int32_t *num_tokens;   /* device int32, or NULL */
+} verify_attn_merge_stacked_args;
+
+int verify_attn_merge_stacked(const verify_attn_merge_stacked_args *args, verify_attn_stream_t stream);
+
 /* Size of the library-owned workspace used by verify_attn_forward_static. */
 #define VERIFY_ATTN_STATIC_WS_BYTES (128u << 20)
 

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     VerifyAttnArgs,
     VerifyAttnDefragArgs,
     VerifyAttnMergeArgs,
+    VerifyAttnMergeStackedArgs,
     VerifyAttnError,
     VerifyAttnParams,
     VerifyAttnPlan,
@@ -25,6 +26,7 @@ from ._binding import (  # noqa: F401
     verify_attn_defrag,
     verify_attn_forward_static,
     verify_attn_gather,
+    verify_attn_merge_stacked,
     verify_attn_merge_states,
     verify_attn_plan,
     verify_attn_reduce,

@@ -70,6 +70,14 @@ class VerifyAttnMergeArgs(ctypes.Structure):
     ]
 
 
+class VerifyAttnMergeStackedArgs(ctypes.Structure):
+    _fields_ = [
+        ("o", _vp), ("lse_states", _vp), ("num_states", _i32), ("num_heads", _i32), ("out", _vp),
+        ("out_stride_tok", _i64), ("out_stride_head", _i64), ("lse", _vp), ("max_tokens", _i64),
+        ("num_tokens", _vp),
+    ]
+
+
 class VerifyAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
@@ -84,7 +92,7 @@ EXPORTS = (
     "verify_attn_reduce",
     "verify_attn_build_tree_mask", "verify_attn_build_tree_mask_device", "verify_attn_status",
     "verify_attn_forward_static", "verify_attn_defrag", "verify_attn_tree_block", "verify_attn_merge_states",
-    "verify_attn_strerror",
+    "verify_attn_merge_stacked", "verify_attn_strerror",
 )
 
 
@@ -114,6 +122,7 @@ def load_library():
             lib.verify_attn_tree_block.argtypes = [P(VerifyAttnPlan), P(VerifyAttnArgs), ctypes.c_int, _vp, _vp,
                                                    _vp, ctypes.c_size_t, _vp]
             lib.verify_attn_merge_states.argtypes = [P(VerifyAttnMergeArgs), _vp]
+            lib.verify_attn_merge_stacked.argtypes = [P(VerifyAttnMergeStackedArgs), _vp]
             lib.verify_attn_strerror.argtypes = [ctypes.c_int]
             lib.verify_attn_strerror.restype = ctypes.c_char_p
             for name in EXPORTS[:-1]:
@@ -203,6 +212,11 @@ def verify_attn_tree_block(plan, args: VerifyAttnArgs, exclude_self: bool, self_
 def verify_attn_merge_states(args: VerifyAttnMergeArgs, stream: int = 0):
     """Two-state LSE merge (asynchronous)."""
     _check(load_library().verify_attn_merge_states(ctypes.byref(args), stream), "verify_attn_merge_states")
+
+
+def verify_attn_merge_stacked(args: VerifyAttnMergeStackedArgs, stream: int = 0):
+    """Stacked R-state LSE merge (asynchronous)."""
+    _check(load_library().verify_attn_merge_stacked(ctypes.byref(args), stream), "verify_attn_merge_stacked")
 
 
 def verify_attn_status(ws_ptr: int, stream: int = 0):

@@ -357,6 +357,33 @@ int verify_attn_merge_states(const verify_attn_merge_args* a, verify_attn_stream
   return VERIFY_ATTN_OK;
 }
 
+int verify_attn_merge_stacked(const verify_attn_merge_stacked_args* a, verify_attn_stream_t stream) {
+  if (!a || !a->o || !a->lse_states || !a->out) return VERIFY_ATTN_EINVAL;
+  if (a->num_states < 1 || a->num_states > 1024 || a->num_heads < 1 || a->num_heads > VERIFY_ATTN_MAX_HEADS ||
+      a->max_tokens < 0)
+    return VERIFY_ATTN_EINVAL;
+  if (!aligned16(a->o) || !aligned16(a->out) || !row_stride_ok(a->out_stride_tok) ||
+      !row_stride_ok(a->out_stride_head))
+    return VERIFY_ATTN_EINVAL;
+  if (a->max_tokens == 0) return VERIFY_ATTN_OK;
+  va::MergeStackedParams p;
+  p.o = a->o;
+  p.lse = a->lse_states;
+  p.num_states = a->num_states;
+  p.out = a->out;
+  p.out_tok = a->out_stride_tok;
+  p.out_head = a->out_stride_head;
+  p.lse_out = a->lse;
+  p.max_tokens = a->max_tokens;
+  p.num_tokens = a->num_tokens;
+  p.num_heads = a->num_heads;
+  if (va::launch_merge_stacked(p, (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return VERIFY_ATTN_CUDA_ERROR;
+  }
+  return VERIFY_ATTN_OK;
+}
+
 int verify_attn_defrag(const verify_attn_defrag_args* a, verify_attn_stream_t stream) {
   if (!a || !a->kv_pool || !a->kv_indices || !a->kv_indptr || !a->dst_begin) return VERIFY_ATTN_EINVAL;
   if (a->batch < 1 || a->budget < 0 || a->pool_slots < 1 || a->pool_slots > INT32_MAX) return VERIFY_ATTN_EINVAL;

@@ -75,7 +75,71 @@ __global__ void __launch_bounds__(kMergeWarps * 32) verify_merge_kernel(const Me
   }
 }
 
+// R states stacked along a leading axis (the KV-sequence shards of one call,
+// gathered from the ranks): m = max_r lse_r, w_r = exp(lse_r - m),
+// out = sum_r w_r o_r / sum_r w_r, lse = m + ln sum_r w_r, rounded to bf16
+// once. Lane r (< R, in chunks of 32) holds state r's weight; the rows are
+// accumulated in fp32 in the order r = 0, 1, ....
+__global__ void __launch_bounds__(kMergeWarps * 32) verify_merge_stacked_kernel(const MergeStackedParams p) {
+  const int lane = threadIdx.x & 31;
+  int64_t tokens = p.max_tokens;
+  if (p.num_tokens) {
+    const int64_t d = *p.num_tokens;
+    tokens = d < 0 ? 0 : (d < tokens ? d : tokens);
+  }
+  const int64_t rows = tokens * p.num_heads;
+  const int64_t state_rows = p.max_tokens * p.num_heads;
+  for (int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5); row < rows;
+       row += (int64_t)gridDim.x * kMergeWarps) {
+    float m = -CUDART_INF_F;
+    for (int r = lane; r < p.num_states; r += 32) m = fmaxf(m, p.lse[(int64_t)r * state_rows + row]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const bool empty = !(m > -CUDART_INF_F);
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    float wsum = 0.f;
+    for (int r0 = 0; r0 < p.num_states; r0 += 32) {
+      const int r_mine = r0 + lane;
+      const float w_mine =
+          (!empty && r_mine < p.num_states) ? expf(p.lse[(int64_t)r_mine * state_rows + row] - m) : 0.f;
+      const int n = p.num_states - r0 < 32 ? p.num_states - r0 : 32;
+      for (int k = 0; k < n; ++k) {
+        const float w = __shfl_sync(0xffffffffu, w_mine, k);
+        if (!(w > 0.f)) continue;   // uniform: every lane holds the same w
+        wsum += w;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.o + ((int64_t)(r0 + k) * state_rows + row) * kDLatent);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 x = bf2(src[lane + 32 * j]);
+          acc[2 * j] = fmaf(w, x.x, acc[2 * j]);
+          acc[2 * j + 1] = fmaf(w, x.y, acc[2 * j + 1]);
+        }
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    const int64_t g = row / p.num_heads, h = row % p.num_heads;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + g * p.out_tok + h * p.out_head);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * j] * inv, acc[2 * j + 1] * inv);
+      dst[lane + 32 * j] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    if (lane == 0 && p.lse_out) p.lse_out[row] = wsum > 0.f ? m + logf(wsum) : -CUDART_INF_F;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_merge_stacked(const MergeStackedParams& p, cudaStream_t stream) {
+  const int64_t rows = p.max_tokens * p.num_heads;
+  int64_t grid = (rows + kMergeWarps - 1) / kMergeWarps;
+  if (grid > 148 * 8) grid = 148 * 8;
+  if (grid < 1) grid = 1;
+  verify_merge_stacked_kernel<<<(unsigned)grid, kMergeWarps * 32, 0, stream>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   const int64_t rows = p.max_tokens * p.num_heads;

@@ -1,6 +1,6 @@
 // Internal interface of the split-verify variant's kernels: the masked
-// tree-block attention (verify_tree_block.cu) and the two-state LSE merge
-// (verify_merge.cu).
+// tree-block attention (verify_tree_block.cu), the two-state LSE merge and
+// the stacked R-state merge of KV-sequence shards (verify_merge.cu).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -48,6 +48,19 @@ struct MergeParams {
   int32_t num_heads;
 };
 
+struct MergeStackedParams {
+  const uint16_t* o;         // bf16 [R, max_tokens, H, 512] contiguous
+  const float* lse;          // [R, max_tokens, H]
+  int32_t num_states;        // R >= 1
+  uint16_t* out;             // bf16 [tokens, H, 512], strides in elements
+  int64_t out_tok, out_head;
+  float* lse_out;            // or null
+  int64_t max_tokens;
+  const int32_t* num_tokens; // or null
+  int32_t num_heads;
+};
+
+cudaError_t launch_merge_stacked(const MergeStackedParams& p, cudaStream_t stream);
 cudaError_t launch_tree_block(const TreeBlockParams& p, int64_t max_tokens, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
