@@ -129,3 +129,58 @@ def test_tree_mask_helper_rejects_malformed(parents):
     with pytest.raises(va.VerifyAttnError) as e:
         va.verify_attn_build_tree_mask(np.asarray(parents, np.int32))
     assert e.value.code == -1
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="uses fake device pointers; host-only check")
+def test_variant_entry_points_reject_bad_arguments_without_launching():
+    """Relocation, tree block and both merges validate before any launch."""
+    lib = va.load_library()
+    P = ctypes.byref
+    d = va.VerifyAttnDefragArgs(kv_pool=16, kv_row_stride=576, pool_slots=100, kv_indices=16, kv_indptr=16,
+                                dst_begin=16, batch=1, budget=4, max_total_kv=10, status=None)
+    for field, bad in (("kv_pool", 8), ("kv_row_stride", 570), ("kv_row_stride", 560), ("batch", 0),
+                       ("budget", -1), ("pool_slots", 0), ("max_total_kv", -1), ("dst_begin", None)):
+        good = getattr(d, field)
+        setattr(d, field, bad)
+        assert lib.verify_attn_defrag(P(d), None) == -1, field
+        setattr(d, field, good)
+    assert lib.verify_attn_defrag(None, None) == -1
+
+    m = va.VerifyAttnMergeArgs(o_a=16, o_a_stride_tok=4096, o_a_stride_head=512, lse_a=16, o_b=16,
+                               o_b_stride_tok=4096, o_b_stride_head=512, lse_b=16, o_b_f32=0, out=16,
+                               out_stride_tok=4096, out_stride_head=512, lse=None, max_tokens=4, num_tokens=None,
+                               num_heads=8)
+    for field, bad in (("o_a", 8), ("out", None), ("lse_b", None), ("o_b_stride_head", 4), ("num_heads", 0),
+                       ("num_heads", 2048), ("max_tokens", -1)):
+        good = getattr(m, field)
+        setattr(m, field, bad)
+        assert lib.verify_attn_merge_states(P(m), None) == -1, field
+        setattr(m, field, good)
+    m.max_tokens = 0                                        # nothing to merge: no launch, success
+    assert lib.verify_attn_merge_states(P(m), None) == 0
+
+    s = va.VerifyAttnMergeStackedArgs(o=16, lse_states=16, num_states=2, num_heads=8, out=16,
+                                      out_stride_tok=4096, out_stride_head=512, lse=None, max_tokens=4,
+                                      num_tokens=None)
+    for field, bad in (("num_states", 0), ("num_states", 1025), ("o", 8), ("out_stride_tok", 100),
+                       ("lse_states", None), ("max_tokens", -2)):
+        good = getattr(s, field)
+        setattr(s, field, bad)
+        assert lib.verify_attn_merge_stacked(P(s), None) == -1, field
+        setattr(s, field, good)
+    s.max_tokens = 0
+    assert lib.verify_attn_merge_stacked(P(s), None) == 0
+
+    plan, ws = va.verify_attn_plan(_params())
+    args = va.VerifyAttnArgs(q_latent=16, q_latent_stride_tok=64 * 512, q_latent_stride_head=512,
+                             q_rope=16, q_rope_stride_tok=64 * 64, q_rope_stride_head=64,
+                             kv_pool=16, kv_row_stride=576, kv_indices=16, kv_indptr=16, qo_indptr=16,
+                             tree_anc=16, batch=1, out=16, out_stride_tok=64 * 512, out_stride_head=512, lse=None)
+    # the tree block needs an LSE output, and an output of one kind or the other
+    assert lib.verify_attn_tree_block(P(plan), P(args), 1, None, None, 256, ws, None) == -1
+    args.lse = 16
+    args.out = None
+    assert lib.verify_attn_tree_block(P(plan), P(args), 1, None, None, 256, ws, None) == -1
+    assert lib.verify_attn_tree_block(P(plan), P(args), 1, None, 8, 256, ws, None) == -1   # misaligned fp32 out
+    assert lib.verify_attn_tree_block(P(plan), P(args), 1, None, 16, 256, ws - 1, None) == -3
