@@ -12,6 +12,10 @@ requests' KV lengths per call / device time per call), whole job over all
 ranks; ``--gpus N`` runs N independent replicas (the path needs no
 collective). ``--impl reference`` times the float64 CPU oracle instead, on a
 bounded sample of the same workload.
+
+``--op defrag`` (KV relocation), ``--op split-verify`` (tree block + dense
+pass + merge) and ``--op sequence-shard`` (the KV split over the ranks, NCCL
+all-gather and stacked merge) print lines of their own on the same workload.
 """
 from __future__ import annotations
 
